@@ -1,0 +1,205 @@
+"""MLA decode over a paged KV cache on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding of libmla (include/mla.h).  It only checks tensors, allocates
+outputs / workspace through PyTorch and passes raw device pointers and the current CUDA
+stream; every step of the computation runs in the library's CUDA kernels.  Importing the
+package fails loudly when libmla.so has not been built: there is no fallback.
+
+Calls (same names as the C-ABI):
+    mla_num_sm_parts(rows_per_kv_head, h_kv=1, device=None)
+    mla_get_metadata(cache_seqlens, rows_per_kv_head, h_kv=1, num_sm_parts=None)
+        -> (tile_md int32 [num_sm_parts, 8], num_splits int32 [batch + 1])
+    mla_workspace_size(batch, num_sm_parts, rows_per_kv_head, h_kv=1)
+    mla_decode_kvcache(q, kvcache, block_table, cache_seqlens, d_v, tile_md, num_splits,
+                       softmax_scale=None, causal=False, ...) -> (out bf16, lse fp32)
+    mla_read_status(workspace, reset=False)
+
+The FlashMLA-style spellings of the usage examples on the pages are provided too:
+get_mla_metadata(cache_seqlens, s_q * h_q // h_kv, h_kv) and
+flash_mla_with_kvcache(q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata,
+num_splits, causal=..., softmax_scale=...).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmla.so")
+
+D_QK = 576
+D_V = 512
+PAGE = 64
+FP8_TOKEN_BYTES = 656
+KV_BF16 = 0
+KV_FP8 = 1
+
+MLA_ERRORS = {
+    -1: "MLA_ERR_NULL_POINTER", -2: "MLA_ERR_MISALIGNED", -3: "MLA_ERR_BAD_DIM", -4: "MLA_ERR_BAD_HEADS",
+    -5: "MLA_ERR_BAD_KV_DTYPE", -6: "MLA_ERR_WORKSPACE", -7: "MLA_ERR_BAD_SHAPE", -8: "MLA_ERR_BAD_PARTS",
+    -9: "MLA_ERR_NO_DEVICE", -100: "MLA_ERR_CUDA",
+}
+
+
+class MLAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {MLA_ERRORS.get(code, code)} ({mla_strerror(code)})")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python attention_mla_get_b200/build.py` "
+                          "(there is no non-CUDA fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    i32, i64, vp, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+    lib.mla_num_sm_parts.argtypes = [i32, i32, i32]
+    lib.mla_num_sm_parts.restype = i32
+    lib.mla_get_metadata.argtypes = [vp, i32, i32, i32, vp, i32, vp, vp]
+    lib.mla_get_metadata.restype = i32
+    lib.mla_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.mla_workspace_size.restype = sz
+    lib.mla_decode_kvcache.argtypes = [vp, vp, i64, vp, i32, vp, i32, i32, i32, i32, i32, vp, i32, vp,
+                                       ctypes.c_float, i32, i32, vp, vp, vp, sz, vp]
+    lib.mla_decode_kvcache.restype = i32
+    lib.mla_read_status.argtypes = [vp, i32, ctypes.POINTER(i32), vp]
+    lib.mla_read_status.restype = i32
+    lib.mla_strerror.argtypes = [i32]
+    lib.mla_strerror.restype = ctypes.c_char_p
+    lib.mla_version.argtypes = []
+    lib.mla_version.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+EXPORTED = ("mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
+            "mla_read_status", "mla_strerror", "mla_version")
+
+
+def mla_strerror(code: int) -> str:
+    return _lib.mla_strerror(int(code)).decode()
+
+
+def mla_version() -> str:
+    return _lib.mla_version().decode()
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise MLAError(code, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def mla_num_sm_parts(rows_per_kv_head: int, h_kv: int = 1, device=None) -> int:
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index or 0
+    n = _lib.mla_num_sm_parts(int(rows_per_kv_head), int(h_kv), int(dev))
+    if n < 1:
+        raise MLAError(n, "mla_num_sm_parts")
+    return n
+
+
+def mla_workspace_size(batch: int, num_sm_parts: int, rows_per_kv_head: int, h_kv: int = 1) -> int:
+    return int(_lib.mla_workspace_size(int(batch), int(num_sm_parts), int(rows_per_kv_head), int(h_kv)))
+
+
+def mla_get_metadata(cache_seqlens: torch.Tensor, rows_per_kv_head: int, h_kv: int = 1,
+                     num_sm_parts: Optional[int] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Tile-scheduler metadata for one decode step (reusable by every layer)."""
+    if cache_seqlens.dtype != torch.int32 or not cache_seqlens.is_cuda or cache_seqlens.dim() != 1:
+        raise ValueError("cache_seqlens must be a 1-D int32 CUDA tensor")
+    cache_seqlens = cache_seqlens.contiguous()
+    batch = cache_seqlens.shape[0]
+    if num_sm_parts is None:
+        num_sm_parts = mla_num_sm_parts(rows_per_kv_head, h_kv, cache_seqlens.device)
+    tile_md = torch.empty((num_sm_parts, 8), dtype=torch.int32, device=cache_seqlens.device)
+    num_splits = torch.empty((batch + 1,), dtype=torch.int32, device=cache_seqlens.device)
+    _check(_lib.mla_get_metadata(_ptr(cache_seqlens), batch, int(rows_per_kv_head), int(h_kv), _ptr(tile_md),
+                                 int(num_sm_parts), _ptr(num_splits), _stream(stream)), "mla_get_metadata")
+    return tile_md, num_splits
+
+
+def mla_decode_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torch.Tensor,
+                       cache_seqlens: torch.Tensor, d_v: int, tile_md: torch.Tensor, num_splits: torch.Tensor,
+                       softmax_scale: Optional[float] = None, causal: bool = False,
+                       kv_dtype: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """MLA decode: returns (out bf16 [b, s_q, h_q, 512], lse fp32 [b, h_q, s_q])."""
+    if q.dtype != torch.bfloat16 or q.dim() != 4 or q.shape[-1] != D_QK:
+        raise ValueError("q must be bf16 [batch, s_q, h_q, 576]")
+    if not q.is_contiguous():
+        q = q.contiguous()
+    b, s_q, h_q, _ = q.shape
+    if kv_dtype is None:
+        kv_dtype = KV_FP8 if kvcache.dtype == torch.uint8 else KV_BF16
+    if kv_dtype == KV_BF16:
+        if kvcache.dtype != torch.bfloat16 or kvcache.shape[1] != PAGE or kvcache.shape[-1] != D_QK:
+            raise ValueError("bf16 kvcache must be [num_blocks, 64, (1,) 576]")
+        h_kv = kvcache.shape[2] if kvcache.dim() == 4 else 1
+    else:
+        if kvcache.dtype != torch.uint8 or kvcache.shape[1] != PAGE or kvcache.shape[-1] != FP8_TOKEN_BYTES:
+            raise ValueError("fp8 kvcache must be uint8 [num_blocks, 64, (1,) 656]")
+        h_kv = kvcache.shape[2] if kvcache.dim() == 4 else 1
+    if not kvcache.is_contiguous():
+        raise ValueError("kvcache must be contiguous")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != b:
+        raise ValueError("block_table must be int32 [batch, max_blocks]")
+    block_table = block_table.contiguous()
+    if softmax_scale is None:
+        softmax_scale = D_QK ** -0.5
+    rows = s_q * h_q // max(1, h_kv)
+    num_sm_parts = tile_md.shape[0]
+    if out is None:
+        out = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    need = mla_workspace_size(b, num_sm_parts, rows, h_kv)
+    if workspace is None:
+        workspace = torch.zeros((max(need, 256),), dtype=torch.uint8, device=q.device)
+    _check(_lib.mla_decode_kvcache(
+        _ptr(q), _ptr(kvcache), kvcache.shape[0], _ptr(block_table), block_table.shape[1], _ptr(cache_seqlens),
+        b, s_q, h_q, h_kv, int(d_v), _ptr(tile_md), num_sm_parts, _ptr(num_splits), float(softmax_scale),
+        1 if causal else 0, int(kv_dtype), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)), "mla_decode_kvcache")
+    return out, lse
+
+
+def mla_read_status(workspace: torch.Tensor, reset: bool = False, stream=None) -> int:
+    v = ctypes.c_int(0)
+    _check(_lib.mla_read_status(_ptr(workspace), 1 if reset else 0, ctypes.byref(v), _stream(stream)),
+           "mla_read_status")
+    return v.value
+
+
+# FlashMLA-style spellings from the pages' usage examples
+def get_mla_metadata(cache_seqlens: torch.Tensor, num_heads_per_head_k: int, num_heads_k: int):
+    return mla_get_metadata(cache_seqlens, num_heads_per_head_k, num_heads_k)
+
+
+def flash_mla_with_kvcache(q, k_cache, block_table, cache_seqlens, head_dim_v, tile_scheduler_metadata,
+                           num_splits, softmax_scale=None, causal=False, is_fp8_kvcache=False):
+    return mla_decode_kvcache(q, k_cache, block_table, cache_seqlens, head_dim_v, tile_scheduler_metadata,
+                              num_splits, softmax_scale=softmax_scale, causal=causal,
+                              kv_dtype=KV_FP8 if is_fp8_kvcache else None)
+
+
+__all__ = [
+    "mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache", "mla_read_status",
+    "mla_strerror", "mla_version", "get_mla_metadata", "flash_mla_with_kvcache", "MLAError", "LIB_PATH",
+    "KV_BF16", "KV_FP8",
+]

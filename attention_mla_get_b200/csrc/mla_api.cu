@@ -1,0 +1,218 @@
+// C-ABI of libmla (declared in include/mla.h): host-side argument checks, workspace
+// partitioning, TMA descriptor encoding and the kernel launches.  No compute happens here.
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/mla.h"
+#include "mla_internal.h"
+
+namespace {
+
+using mla::kDqk;
+using mla::kDv;
+using mla::kPage;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr size_t kHeaderBytes = 256;
+constexpr int kMaxRows = 4096;
+
+struct WorkspaceLayout {
+  size_t lse_off, o_off, total;
+};
+
+WorkspaceLayout workspace_layout(int batch, int parts, int rows) {
+  const size_t splits = static_cast<size_t>(batch) + static_cast<size_t>(parts);
+  WorkspaceLayout w;
+  w.lse_off = kHeaderBytes;
+  w.o_off = round_up(w.lse_off + splits * rows * sizeof(float), 256);
+  w.total = w.o_off + splits * rows * kDv * sizeof(float);
+  return w;
+}
+
+int rows_per_cta_for(int rows) { return rows <= 16 ? 16 : (rows <= 32 ? 32 : 64); }
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_version(void) { return "0.1.0"; }
+
+const char* mla_strerror(int code) {
+  switch (code) {
+    case MLA_OK: return "success";
+    case MLA_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case MLA_ERR_MISALIGNED: return "q, kvcache, out and workspace must be 16-byte aligned, lse 4-byte aligned";
+    case MLA_ERR_BAD_DIM: return "d_v must be 512 (V is the first 512 of the 576 cached dims)";
+    case MLA_ERR_BAD_HEADS: return "h_kv must be 1, h_q >= 1 and h_q % h_kv == 0";
+    case MLA_ERR_BAD_KV_DTYPE: return "kv_dtype must be MLA_KV_BF16 or MLA_KV_FP8";
+    case MLA_ERR_WORKSPACE: return "workspace is smaller than mla_workspace_size()";
+    case MLA_ERR_BAD_SHAPE: return "bad shape: batch, s_q, num_blocks, max_blocks must be >= 1, "
+                                   "s_q*h_q <= 4096 and num_blocks*64 < 2^31";
+    case MLA_ERR_BAD_PARTS: return "num_sm_parts must be >= 1";
+    case MLA_ERR_NO_DEVICE: return "CUDA device query failed";
+    case MLA_ERR_CUDA: return "a CUDA call failed";
+    default: return "unknown libmla error code";
+  }
+}
+
+int mla_num_sm_parts(int rows_per_kv_head, int h_kv, int device) {
+  if (h_kv != 1) return MLA_ERR_BAD_HEADS;
+  if (rows_per_kv_head < 1 || rows_per_kv_head > kMaxRows) return MLA_ERR_BAD_SHAPE;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms < 1)
+    return MLA_ERR_NO_DEVICE;
+  const int g = mla::row_groups_for(rows_per_kv_head);
+  const int parts = sms / (h_kv * g);
+  return parts < 1 ? 1 : parts;
+}
+
+size_t mla_workspace_size(int batch, int num_sm_parts, int rows_per_kv_head, int h_kv) {
+  if (batch < 1 || num_sm_parts < 1 || h_kv != 1 || rows_per_kv_head < 1 || rows_per_kv_head > kMaxRows) return 0;
+  return workspace_layout(batch, num_sm_parts, rows_per_kv_head).total;
+}
+
+int mla_get_metadata(const int32_t* cache_seqlens, int batch, int rows_per_kv_head, int h_kv, int32_t* tile_md,
+                     int num_sm_parts, int32_t* num_splits, void* stream) {
+  if (!cache_seqlens || !tile_md || !num_splits) return MLA_ERR_NULL_POINTER;
+  if (batch < 1 || rows_per_kv_head < 1 || rows_per_kv_head > kMaxRows) return MLA_ERR_BAD_SHAPE;
+  if (h_kv != 1) return MLA_ERR_BAD_HEADS;
+  if (num_sm_parts < 1) return MLA_ERR_BAD_PARTS;
+  const int e = mla::launch_scheduler(cache_seqlens, batch, num_sm_parts, tile_md, num_splits,
+                                      static_cast<cudaStream_t>(stream));
+  return e == 0 ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, const int32_t* block_table,
+                       int max_blocks, const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                       int d_v, const int32_t* tile_md, int num_sm_parts, const int32_t* num_splits,
+                       float softmax_scale, int causal, int kv_dtype, void* out, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  // ---- argument checks (nothing is enqueued before they all pass) ----
+  if (!q || !kvcache || !block_table || !cache_seqlens || !tile_md || !num_splits || !out || !lse || !workspace)
+    return MLA_ERR_NULL_POINTER;
+  if (!aligned(q, 16) || !aligned(kvcache, 16) || !aligned(out, 16) || !aligned(workspace, 16) || !aligned(lse, 4))
+    return MLA_ERR_MISALIGNED;
+  if (d_v != kDv) return MLA_ERR_BAD_DIM;
+  if (h_kv != 1 || h_q < 1 || h_q % h_kv != 0) return MLA_ERR_BAD_HEADS;
+  if (kv_dtype != MLA_KV_BF16 && kv_dtype != MLA_KV_FP8) return MLA_ERR_BAD_KV_DTYPE;
+  if (batch < 1 || s_q < 1 || num_blocks < 1 || max_blocks < 1) return MLA_ERR_BAD_SHAPE;
+  const long long rows_ll = static_cast<long long>(s_q) * h_q / h_kv;
+  if (rows_ll > kMaxRows) return MLA_ERR_BAD_SHAPE;
+  if (num_blocks * kPage >= (1ll << 31)) return MLA_ERR_BAD_SHAPE;
+  if (num_sm_parts < 1) return MLA_ERR_BAD_PARTS;
+  const int rows = static_cast<int>(rows_ll);
+  const WorkspaceLayout wl = workspace_layout(batch, num_sm_parts, rows);
+  if (workspace_bytes < wl.total) return MLA_ERR_WORKSPACE;
+
+  EncodeTiledFn encode = encode_fn();
+  if (!encode) return MLA_ERR_CUDA;
+  const int rg = rows_per_cta_for(rows);
+
+  // q as a 3-D tensor {576 dims, rows, batch}; one box = 64 dims x rg rows of one request
+  CUtensorMap tm_q, tm_kv;
+  {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(batch)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDqk) * 2, static_cast<cuuint64_t>(kDqk) * 2 * rows};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rg), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  if (kv_dtype == MLA_KV_BF16) {
+    // the cache as 2-D {576 dims, num_blocks * 64 tokens}; one box = 64 dims x one page
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(num_blocks) * kPage};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDqk) * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    if (encode(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kvcache), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  } else {
+    // FP8 tokens as 2-D bytes {656, num_blocks * 64}; one box = 656 bytes would exceed the
+    // 256-element box limit, so the kernel reads 4 boxes of 164 bytes... see mla_decode_fp8.cu
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kFp8TokenBytes), static_cast<cuuint64_t>(num_blocks) * kPage};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kFp8TokenBytes)};
+    cuuint32_t box[2] = {128, 64};
+    cuuint32_t estr[2] = {1, 1};
+    if (encode(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(kvcache), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  mla::DecodeParams p{};
+  p.block_table = block_table;
+  p.cache_seqlens = cache_seqlens;
+  p.tile_md = tile_md;
+  p.num_splits = num_splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.lse_part = reinterpret_cast<float*>(ws + wl.lse_off);
+  p.o_part = reinterpret_cast<float*>(ws + wl.o_off);
+  p.status = reinterpret_cast<int*>(ws);
+  p.kv_raw = static_cast<const uint8_t*>(kvcache);
+  p.max_blocks = max_blocks;
+  p.batch = batch;
+  p.num_sm_parts = num_sm_parts;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.rows = rows;
+  p.row_groups = (rows + rg - 1) / rg;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int e = kv_dtype == MLA_KV_BF16 ? mla::launch_decode_bf16(tm_q, tm_kv, p, rg, st)
+                                  : mla::launch_decode_fp8(tm_q, tm_kv, p, st);
+  if (e != 0) return MLA_ERR_CUDA;
+
+  mla::CombineParams cp{};
+  cp.num_splits = num_splits;
+  cp.o_part = p.o_part;
+  cp.lse_part = p.lse_part;
+  cp.out = p.out;
+  cp.lse = lse;
+  cp.batch = batch;
+  cp.s_q = s_q;
+  cp.h_q = h_q;
+  cp.rows = rows;
+  e = mla::launch_combine(cp, st);
+  return e == 0 ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_read_status(void* workspace, int reset, int* status, void* stream) {
+  if (!workspace || !status) return MLA_ERR_NULL_POINTER;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  *status = v;
+  if (reset && cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+}  // extern "C"

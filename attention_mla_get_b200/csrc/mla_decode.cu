@@ -1,0 +1,605 @@
+// Split-KV MLA decode main kernel for sm_100a (bf16 paged KV cache).
+//
+// Problem (FlashMLA pages: mha_fwd_kvcache_mla / run_mha_fwd_splitkv_mla<bf16, 576> in the
+// "flash_api.cpp" excerpt, mmssai.com page; 64-token pages addressed by block_table,
+// kdjingpai.com page; query folding q.view(b, s_q, h_kv, ngroups, d).transpose(2, 3),
+// deepseekonline.chat page): for each request, R = s_q*h_q query rows attend to one shared
+// latent KV of 576 dims; V is the first 512 dims of the same cached vector.
+//
+// Design (B200-native, "swap-AB"): the KV tile is the large operand, so it is the M side
+// of every tcgen05 MMA and the query rows are the N side:
+//   S^T [128 tokens x RG rows]  = K_tile[128 x 576]  . Q^T[576 x RG]      (fp32 in TMEM)
+//   O^T [512 dims  x RG rows] += V_tile^T[512 x 128] . P^T[128 x RG]      (fp32 in TMEM)
+// One CTA carries RG <= 64 query rows (R = 128 / 256 uses 2 / 4 CTAs on the same pages),
+// so O^T needs only 4*RG TMEM columns and the whole 512-dim output stays in TMEM.
+// A step covers 128 tokens (two 64-token pages).  Pages are TMA-loaded through the block
+// table in 64x64 boxes (the 9-boxes-per-page split on the wmrh.cn page, "内存访问优化策略")
+// into 32 KB ring slots (128 tokens x 128 dims, 128-byte swizzle).  The same slot is read
+// K-major by QK^T and MN-major (as V^T) by PV, so V is never transposed.
+//
+// Roles (192 threads):  warps 0-3 online softmax + epilogue (thread = token lane of S^T,
+// then dim lane of O^T), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner.
+// Online softmax keeps a per-row running reference max (log2 units) and rescales O^T in
+// TMEM only when a block max exceeds it by more than kTau (the running-max-and-scale
+// idea of the wmrh.cn page, "跷跷板调度算法" paragraph); P^T is written to shared memory
+// as bf16, the row sums use the unrounded fp32 P.
+//
+// Two load schedules:
+//   RETAIN (RG = 16): K(t) slots 0-3 are kept and reused as V(t); QK(t) -> softmax(t) ->
+//                     PV(t) in order.  One HBM read, one shared-memory fill per byte.
+//   RELOAD (RG >= 32): K(t+1) is multiplied while softmax(t) runs; V(t) is reloaded
+//                     (an L2 hit) after K(t+1) because the ring cannot hold both steps.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "mla_internal.h"
+#include "mla_ptx.cuh"
+
+namespace mla {
+
+namespace {
+
+constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units (P <= 2^8)
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int RG, bool RETAIN>
+struct Cfg {
+  static constexpr int kSlotBytes = 32768;   // 128 tokens x 128 dims bf16
+  static constexpr int kAtomColBytes = 16384;// 128 tokens x 64 dims (one swizzle column)
+  static constexpr int kPageBoxBytes = 8192; // 64 tokens x 64 dims: one TMA box
+  static constexpr int kQAtomBytes = RG * 128;
+  static constexpr int kQBytes = 9 * kQAtomBytes;
+  static constexpr int kPRowBytes = RG * 2;  // one token row of P^T (MN-major, rows contiguous)
+  static constexpr int kPBytes = 128 * kPRowBytes;
+  static constexpr int kNumP = (RG == 64) ? 1 : 2;
+  static constexpr int kNumSlots = RETAIN ? 6 : (RG == 64 ? 4 : 5);
+  static constexpr int kTmemCols = RG == 16 ? 128 : (RG == 32 ? 256 : 512);
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffP = kOffQ + kQBytes;
+  static constexpr int kOffSlots = kOffP + kNumP * kPBytes;
+  static constexpr int kOffMisc = kOffSlots + kNumSlots * kSlotBytes;
+  static constexpr int kMiscBytes = 3072;
+  static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kPSwzMask = RG / 8 - 1;                // (row bytes / 16) - 1
+  static constexpr uint32_t kPLayout = RG == 64 ? kSwizzle128 : (RG == 32 ? kSwizzle64 : kSwizzle32);
+  static constexpr uint32_t kIdescQK = idesc_bf16(128, RG, false, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16(128, RG, true, true);
+  static constexpr int kColO = 0;       // 4 blocks of RG columns: O^T dims 128j..128j+127
+  static constexpr int kColS = 4 * RG;  // 2 buffers of RG columns: S^T
+  static constexpr int kNOut = RG == 64 ? 2 : 1;  // columns per lane after a warp reduce-scatter
+  static constexpr int kSlotsPerStep = RETAIN ? 5 : 9;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kQBytes % 1024 == 0 && kPBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+};
+
+// barrier indices in the misc area
+enum : int {
+  kBarSlotFull = 0,    // [6]
+  kBarSlotEmpty = 6,   // [6]
+  kBarSFull = 12,      // [2]
+  kBarSEmpty = 14,     // [2]
+  kBarPFull = 16,      // [2]
+  kBarPEmpty = 18,     // [2]
+  kBarQFull = 20,
+  kBarQEmpty = 21,
+  kBarOFull = 22,
+  kBarOEmpty = 23,
+  kBarDrain = 24,
+  kNumBars = 25,
+};
+
+__device__ __forceinline__ int blocks_of(int L) { return L > 0 ? (L + kBlockTokens - 1) / kBlockTokens : 0; }
+
+// Walks the chunks of one scheduler part: (request b, blocks [c0, c1), split index).
+struct ChunkWalk {
+  int b, blk, split, end_b, end_blk;
+  __device__ ChunkWalk(const DecodeParams& p, int part) {
+    const int32_t* md = p.tile_md + part * kMdInts;
+    b = md[0];
+    blk = md[1];
+    end_b = md[2];
+    end_blk = md[3];
+    split = md[4];
+  }
+  __device__ bool next(const DecodeParams& p, int& cb, int& c0, int& c1, int& csplit) {
+    while (b < end_b || (b == end_b && blk < end_blk)) {
+      const int n = blocks_of(p.cache_seqlens[b]);
+      const int stop = (b == end_b) ? end_blk : n;
+      cb = b;
+      c0 = blk;
+      c1 = stop;
+      csplit = split;
+      ++b;
+      blk = 0;
+      if (b <= p.batch) split = p.num_splits[b];
+      if (stop > c0) return true;
+    }
+    return false;
+  }
+};
+
+// Drain wait used only after an abort: bounded, does not look at the abort flag.
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) return;
+  }
+}
+
+// Lane 0 waits, the warp learns the outcome.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& wc, int lane) {
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(bar, parity, wc) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Warp reduce-scatter over the 32 token lanes of N column values.  Afterwards lane l holds
+// the warp-wide reduction of column col_of(l, i) in v[i], i < max(1, N / 32).
+template <int N, bool MAX>
+__device__ __forceinline__ void reduce_scatter(float* v, int lane) {
+#pragma unroll
+  for (int r = 0; r < 5; ++r) {
+    const int o = 16 >> r;
+    const int n = N >> r;
+    if (n > 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < n / 2; ++i) {
+        const float keep = upper ? v[i + n / 2] : v[i];
+        const float send = upper ? v[i] : v[i + n / 2];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+        v[i] = MAX ? fmaxf(keep, recv) : keep + recv;
+      }
+    } else {
+      const float recv = __shfl_xor_sync(0xffffffffu, v[0], o);
+      v[0] = MAX ? fmaxf(v[0], recv) : v[0] + recv;
+    }
+  }
+}
+
+template <int RG>
+__device__ __forceinline__ int col_of(int lane, int i) {
+  if constexpr (RG == 64) return 2 * lane + i;
+  else if constexpr (RG == 32) return lane;
+  else return lane >> 1;
+}
+
+template <int RG, bool RETAIN>
+__global__ void __launch_bounds__(192, 1)
+    mla_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                           const DecodeParams p) {
+  using C = Cfg<RG, RETAIN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::kOffQ;
+  const uint32_t sP = sbase + C::kOffP;
+  const uint32_t sSlots = sbase + C::kOffSlots;
+  uint8_t* misc = smem + C::kOffMisc;
+  const uint32_t sBars = smem_u32(misc);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 260);
+  float* red = reinterpret_cast<float*>(misc + 512);        // [4][64]
+  float* m_sm = reinterpret_cast<float*>(misc + 1536);      // [64]
+  float* alpha_sm = reinterpret_cast<float*>(misc + 1792);  // [64]
+  float* inv_sm = reinterpret_cast<float*>(misc + 2048);    // [64]
+  auto bar = [&](int i) -> uint32_t { return sBars + 8u * static_cast<uint32_t>(i); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int part = blockIdx.x;
+  const int rg = blockIdx.y;  // row group
+  const WaitCtl wc{abort_flag, p.status, kStatusWaitTimeout};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 6; ++i) {
+      mbar_init(bar(kBarSlotFull + i), 1);
+      mbar_init(bar(kBarSlotEmpty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarSEmpty + i), 4);
+      mbar_init(bar(kBarPFull + i), 4);
+      mbar_init(bar(kBarPEmpty + i), 1);
+    }
+    mbar_init(bar(kBarQFull), 1);
+    mbar_init(bar(kBarQEmpty), 1);
+    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarOEmpty), 4);
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kv);
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  // Zero the ring once: a page half that is never loaded then holds finite values.
+  for (int i = threadIdx.x; i < C::kNumSlots * C::kSlotBytes / 16; i += blockDim.x)
+    st_shared_v4(sSlots + 16u * i, 0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  pdl_launch_dependents();
+
+  if (warp == 4) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+      // dims < 512 are read again (V reload or the other row groups): keep them in L2
+      const uint64_t pol_k = (!RETAIN || p.row_groups > 1) ? pol_keep : pol_stream;
+      const uint64_t pol_v = p.row_groups > 1 ? pol_keep : pol_stream;
+      uint32_t g = 0;  // slot fills issued
+      int last_use[6] = {-1, -1, -1, -1, -1, -1};
+      int q_fills = 0;
+      bool ok = true;
+      ChunkWalk walk(p, part);
+      int b, c0, c1, split;
+      auto fill = [&](int dims0, int natoms, int pA, int pB, bool hasB, uint64_t pol) -> bool {
+        const int s = static_cast<int>(g % C::kNumSlots);
+        const uint32_t use = g / C::kNumSlots;
+        if (!mbar_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
+        const uint32_t bytes = static_cast<uint32_t>(natoms * (hasB ? 2 : 1) * C::kPageBoxBytes);
+        mbar_arrive_expect_tx(bar(kBarSlotFull + s), bytes);
+        const uint32_t dst = sSlots + static_cast<uint32_t>(s) * C::kSlotBytes;
+        for (int a = 0; a < natoms; ++a) {
+          tma_load_2d(dst + a * C::kAtomColBytes, &tm_kv, dims0 + 64 * a, pA * kPage, bar(kBarSlotFull + s), pol);
+          if (hasB)
+            tma_load_2d(dst + a * C::kAtomColBytes + C::kPageBoxBytes, &tm_kv, dims0 + 64 * a, pB * kPage,
+                        bar(kBarSlotFull + s), pol);
+        }
+        last_use[s] = static_cast<int>(use);
+        ++g;
+        return true;
+      };
+      while (ok && walk.next(p, b, c0, c1, split)) {
+        const int L = p.cache_seqlens[b];
+        const int npages = (L + kPage - 1) / kPage;
+        const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
+        if (!mbar_wait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(bar(kBarQFull), 9u * C::kQAtomBytes);
+        for (int a = 0; a < 9; ++a) tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, 64 * a, rg * RG, b, bar(kBarQFull));
+        ++q_fills;
+        int prevA = 0, prevB = 0;
+        bool prevHasB = false;
+        for (int t = 0; ok && t < c1 - c0; ++t) {
+          const int blk = c0 + t;
+          const int pA = bt[2 * blk];
+          const bool hasB = 2 * blk + 1 < npages;
+          const int pB = hasB ? bt[2 * blk + 1] : 0;
+          for (int ks = 0; ok && ks < 4; ++ks) ok = fill(128 * ks, 2, pA, pB, hasB, pol_k);
+          if (ok) ok = fill(512, 1, pA, pB, hasB, pol_stream);
+          if (!RETAIN && t > 0)
+            for (int vs = 0; ok && vs < 4; ++vs) ok = fill(128 * vs, 2, prevA, prevB, prevHasB, pol_v);
+          prevA = pA;
+          prevB = pB;
+          prevHasB = hasB;
+        }
+        if (!RETAIN)
+          for (int vs = 0; ok && vs < 4; ++vs) ok = fill(128 * vs, 2, prevA, prevB, prevHasB, pol_v);
+      }
+      if (*abort_flag) {
+        // let every copy this warp started land before the CTA may exit
+        for (int s = 0; s < C::kNumSlots; ++s)
+          if (last_use[s] >= 0) mbar_wait_drain(bar(kBarSlotFull + s), static_cast<uint32_t>(last_use[s]) & 1u);
+        if (q_fills > 0) mbar_wait_drain(bar(kBarQFull), static_cast<uint32_t>(q_fills - 1) & 1u);
+      }
+    }
+  } else if (warp == 5) {
+    // ================================ MMA issuer ==================================
+    if (lane == 0) {
+      uint32_t g = 0;  // slot fills consumed
+      uint32_t u = 0;  // global step counter (S / P buffers)
+      int chunk = 0;
+      bool ok = true;
+      ChunkWalk walk(p, part);
+      int b, c0, c1, split;
+      uint32_t gK_prev = 0;
+      auto do_pv = [&](int t, uint32_t uu, uint32_t gK) -> bool {
+        const int pb = static_cast<int>(uu % C::kNumP);
+        if (!mbar_wait(bar(kBarPFull + pb), (uu / C::kNumP) & 1u, wc)) return false;
+        if (t == 0 && !mbar_wait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t pbase = sP + static_cast<uint32_t>(pb) * C::kPBytes;
+        for (int vs = 0; vs < 4; ++vs) {
+          uint32_t s;
+          if (RETAIN) {
+            s = (gK + vs) % C::kNumSlots;
+          } else {
+            s = g % C::kNumSlots;
+            if (!mbar_wait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) return false;
+            ++g;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + C::kColO + vs * RG;
+          const uint32_t vbase = sSlots + s * C::kSlotBytes;
+#pragma unroll
+          for (int kt = 0; kt < 8; ++kt) {
+            const uint64_t adesc = smem_desc(vbase + kt * 2048, C::kAtomColBytes, 1024, kSwizzle128);
+            const uint64_t bdesc = smem_desc(pbase + kt * 16 * C::kPRowBytes, 16 * 8 * C::kPRowBytes,
+                                             8 * C::kPRowBytes, C::kPLayout);
+            umma_bf16(d, adesc, bdesc, C::kIdescPV, (t == 0 && kt == 0) ? 0u : 1u);
+          }
+          umma_commit(bar(kBarSlotEmpty + s));
+        }
+        umma_commit(bar(kBarPEmpty + pb));
+        return true;
+      };
+      while (ok && walk.next(p, b, c0, c1, split)) {
+        const int n = c1 - c0;
+        if (!mbar_wait(bar(kBarQFull), chunk & 1, wc)) break;
+        for (int t = 0; ok && t < n; ++t) {
+          const int sb = static_cast<int>(u & 1u);
+          if (!mbar_wait(bar(kBarSEmpty + sb), ((u >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + C::kColS + sb * RG;
+          const uint32_t gK = g;
+          for (int ks = 0; ks < 5; ++ks) {
+            const uint32_t s = g % C::kNumSlots;
+            if (!mbar_wait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t kbase = sSlots + s * C::kSlotBytes;
+            const int nk = ks < 4 ? 8 : 4;
+            for (int kk = 0; kk < nk; ++kk) {
+              const uint32_t a = kbase + (kk >> 2) * C::kAtomColBytes + (kk & 3) * 32;
+              const uint32_t bq = sQ + (2 * ks + (kk >> 2)) * C::kQAtomBytes + (kk & 3) * 32;
+              umma_bf16(d, smem_desc(a, 16, 1024, kSwizzle128), smem_desc(bq, 16, 1024, kSwizzle128), C::kIdescQK,
+                        (ks | kk) != 0 ? 1u : 0u);
+            }
+            if (!RETAIN || ks == 4) umma_commit(bar(kBarSlotEmpty + s));
+            ++g;
+          }
+          if (!ok) break;
+          umma_commit(bar(kBarSFull + sb));
+          if (t == n - 1) umma_commit(bar(kBarQEmpty));
+          if (RETAIN) {
+            ok = do_pv(t, u, gK);
+          } else if (t > 0) {
+            ok = do_pv(t - 1, u - 1, gK_prev);
+          }
+          gK_prev = gK;
+          ++u;
+        }
+        if (!ok) break;
+        if (!RETAIN) ok = do_pv(n - 1, u - 1, gK_prev);
+        if (!ok) break;
+        umma_commit(bar(kBarOFull));
+        ++chunk;
+      }
+      // every MMA this thread issued is complete before TMEM is released
+      umma_commit(bar(kBarDrain));
+      mbar_wait_drain(bar(kBarDrain), 0);
+    }
+  } else {
+    // ============================ softmax + epilogue ==============================
+    const int tid = threadIdx.x;  // 0..127: token lane of S^T, dim lane of O^T
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float NEG_INF = -CUDART_INF_F;
+    float m_ref = NEG_INF;  // thread c < RG: reference max of row c (log2 units)
+    float lsum[C::kNOut];
+#pragma unroll
+    for (int i = 0; i < C::kNOut; ++i) lsum[i] = 0.f;
+    uint32_t u = 0;
+    uint32_t gchunk = 0;  // slot fills before the current chunk
+    int chunk = 0;
+    bool fail = false;
+    const int R = p.rows;
+    ChunkWalk walk(p, part);
+    int b, c0, c1, split;
+    while (walk.next(p, b, c0, c1, split)) {
+      const int L = p.cache_seqlens[b];
+      const int n = c1 - c0;
+      const bool single = (p.num_splits[b + 1] - p.num_splits[b]) == 1;
+      const int row0 = rg * RG;
+      bool aborted = false;
+      for (int t = 0; t < n; ++t) {
+        const int t0 = (c0 + t) * kBlockTokens;
+        const int j = t0 + tid;
+        const int sb = static_cast<int>(u & 1u);
+        bool ok = warp_wait(bar(kBarSFull + sb), (u >> 1) & 1u, wc, lane);
+        float x[RG];
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < RG; c += 16) tmem_ld16(tmem + lane_base + C::kColS + sb * RG + c, x + c);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarSEmpty + sb));
+        // scale into log2 units and mask: key j is visible to row r iff j < L and, when causal,
+        // j <= L - s_q + r / h_q (the query block sits at the end of the cache).  With
+        // i0 = j - L + s_q that is r / h_q >= i0, i.e. r >= i0 * h_q, i.e. c >= cmin.
+        int cmin = -(1 << 30);
+        if (p.causal) {
+          const int i0 = j - L + p.s_q;
+          if (i0 > 0) cmin = i0 * p.h_q - row0;
+        }
+        if (j >= L) cmin = 1 << 30;
+#pragma unroll
+        for (int c = 0; c < RG; ++c) x[c] = (c >= cmin) ? x[c] * p.scale_log2 : NEG_INF;
+        float v[RG];
+#pragma unroll
+        for (int c = 0; c < RG; ++c) v[c] = x[c];
+        reduce_scatter<RG, true>(v, lane);
+#pragma unroll
+        for (int i = 0; i < C::kNOut; ++i) red[warp * 64 + col_of<RG>(lane, i)] = v[i];
+        if (named_bar_any(1, 128, !ok || fail)) { aborted = true; break; }
+        bool need = false;
+        if (tid < RG) {
+          const float bm = fmaxf(fmaxf(red[tid], red[64 + tid]), fmaxf(red[128 + tid], red[192 + tid]));
+          float alpha = 1.f;
+          float m_new = m_ref;
+          if (bm > m_ref + kTau || (m_ref == NEG_INF && bm != NEG_INF)) {
+            m_new = bm;
+            alpha = (m_ref == NEG_INF) ? 0.f : ex2(m_ref - m_new);
+          }
+          need = (alpha != 1.f) && (t > 0);
+          m_ref = m_new;
+          m_sm[tid] = (m_new == NEG_INF) ? 0.f : m_new;
+          alpha_sm[tid] = alpha;
+        }
+        const bool rescale = named_bar_any(1, 128, need);
+#pragma unroll
+        for (int c = 0; c < RG; c += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(m_sm + c);
+          x[c + 0] = ex2(x[c + 0] - m4.x);
+          x[c + 1] = ex2(x[c + 1] - m4.y);
+          x[c + 2] = ex2(x[c + 2] - m4.z);
+          x[c + 3] = ex2(x[c + 3] - m4.w);
+        }
+#pragma unroll
+        for (int c = 0; c < RG; ++c) v[c] = x[c];
+        reduce_scatter<RG, false>(v, lane);
+#pragma unroll
+        for (int i = 0; i < C::kNOut; ++i) lsum[i] = lsum[i] * alpha_sm[col_of<RG>(lane, i)] + v[i];
+        // P^T row of this token (bf16), once PV(u - kNumP) has released the buffer
+        const int pb = static_cast<int>(u % C::kNumP);
+        if (u >= static_cast<uint32_t>(C::kNumP))
+          ok &= warp_wait(bar(kBarPEmpty + pb), ((u - C::kNumP) / C::kNumP) & 1u, wc, lane);
+        {
+          const uint32_t prow = static_cast<uint32_t>(tid) * C::kPRowBytes;
+          const uint32_t pbase = sP + static_cast<uint32_t>(pb) * C::kPBytes;
+#pragma unroll
+          for (int q = 0; q < RG / 8; ++q) {
+            uint32_t off = prow + 16u * q;
+            off ^= ((off >> 7) & C::kPSwzMask) << 4;
+            st_shared_v4(pbase + off, pack_bf16x2(x[8 * q + 0], x[8 * q + 1]), pack_bf16x2(x[8 * q + 2], x[8 * q + 3]),
+                         pack_bf16x2(x[8 * q + 4], x[8 * q + 5]), pack_bf16x2(x[8 * q + 6], x[8 * q + 7]));
+          }
+        }
+        if (rescale) {
+          // O^T *= alpha per row, after PV(u - 1) has finished
+          const uint32_t up = u - 1;
+          ok &= warp_wait(bar(kBarPEmpty + up % C::kNumP), (up / C::kNumP) & 1u, wc, lane);
+          tc_fence_after();
+#pragma unroll
+          for (int vs = 0; vs < 4; ++vs) {
+#pragma unroll
+            for (int c = 0; c < RG; c += 16) {
+              float o[16];
+              const uint32_t ta = tmem + lane_base + C::kColO + vs * RG + c;
+              tmem_ld16(ta, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] *= alpha_sm[c + e];
+              tmem_st16(ta, o);
+            }
+          }
+          tmem_wait_st();
+        }
+        if (t0 + kBlockTokens > L) {
+          // tail step: zero the V rows of tokens past the end (their cache slots may hold NaN,
+          // and 0 * NaN would poison O)
+          for (int vs = 0; vs < 4; ++vs) {
+            const uint32_t gv = RETAIN ? gchunk + 5u * t + vs
+                                       : gchunk + 5u * static_cast<uint32_t>(min(t + 2, n)) + 4u * t + vs;
+            const uint32_t s = gv % C::kNumSlots;
+            ok &= warp_wait(bar(kBarSlotFull + s), (gv / C::kNumSlots) & 1u, wc, lane);
+            if (j >= L) {
+              const uint32_t rowaddr = sSlots + s * C::kSlotBytes + static_cast<uint32_t>(tid) * 128u;
+#pragma unroll
+              for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) st_shared_v4(rowaddr + a * C::kAtomColBytes + 16u * q, 0u, 0u, 0u, 0u);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarPFull + pb));
+        fail |= !ok;
+        ++u;
+      }
+      if (aborted) break;
+      // ------------------------------- epilogue ---------------------------------
+#pragma unroll
+      for (int i = 0; i < C::kNOut; ++i) red[warp * 64 + col_of<RG>(lane, i)] = lsum[i];
+      if (named_bar_any(1, 128, fail)) break;
+      if (tid < RG) {
+        const float l = red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid];
+        const int row = row0 + tid;
+        const float lse_val = l > 0.f ? (m_ref + log2f(l)) * kLn2 : NEG_INF;
+        inv_sm[tid] = l > 0.f ? 1.f / l : 0.f;
+        if (row < R) {
+          if (single)
+            p.lse[(static_cast<long long>(b) * p.h_q + row % p.h_q) * p.s_q + row / p.h_q] = lse_val;
+          else
+            p.lse_part[static_cast<long long>(split) * R + row] = lse_val;
+        }
+        m_ref = NEG_INF;
+      }
+#pragma unroll
+      for (int i = 0; i < C::kNOut; ++i) lsum[i] = 0.f;
+      named_bar_sync(1, 128);
+      const bool ok = warp_wait(bar(kBarOFull), chunk & 1, wc, lane);
+      fail |= !ok;
+      tc_fence_after();
+#pragma unroll
+      for (int vs = 0; vs < 4; ++vs) {
+        const int dim = vs * 128 + tid;
+#pragma unroll
+        for (int c = 0; c < RG; c += 16) {
+          float o[16];
+          tmem_ld16(tmem + lane_base + C::kColO + vs * RG + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int row = row0 + c + e;
+            if (row < R) {
+              const float val = o[e] * inv_sm[c + e];
+              if (single)
+                p.out[(static_cast<long long>(b) * R + row) * kDv + dim] = __float2bfloat16_rn(val);
+              else
+                p.o_part[(static_cast<long long>(split) * R + row) * kDv + dim] = val;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarOEmpty));
+      gchunk += static_cast<uint32_t>(C::kSlotsPerStep * n);
+      ++chunk;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int RG, bool RETAIN>
+int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, cudaStream_t stream) {
+  using C = Cfg<RG, RETAIN>;
+  auto kern = mla_decode_bf16_kernel<RG, RETAIN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  dim3 grid(p.num_sm_parts, p.row_groups, 1);
+  kern<<<grid, 192, C::kSmemBytes, stream>>>(tm_q, tm_kv, p);
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, int rows_per_cta,
+                       cudaStream_t stream) {
+  switch (rows_per_cta) {
+    case 16: return launch_impl<16, true>(tm_q, tm_kv, p, stream);
+    case 32: return launch_impl<32, false>(tm_q, tm_kv, p, stream);
+    case 64: return launch_impl<64, false>(tm_q, tm_kv, p, stream);
+    default: return static_cast<int>(cudaErrorInvalidValue);
+  }
+}
+
+}  // namespace mla

@@ -1,0 +1,68 @@
+// Internal declarations shared by the C-ABI layer (mla_api.cu) and the kernels.
+// Nothing here is part of the public interface in include/mla.h.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace mla {
+
+constexpr int kDqk = 576;          // 512 latent (NoPE) + 64 RoPE dims per cached token
+constexpr int kDv = 512;           // V = first 512 dims of the cached vector
+constexpr int kPage = 64;          // tokens per KV page
+constexpr int kBlockTokens = 128;  // scheduling unit: two pages, one main-loop step
+constexpr int kFixedSplitCost = 2; // scheduler: cost of opening a chunk, in blocks
+constexpr int kMdInts = 8;         // ints per tile-scheduler metadata row
+constexpr int kRowsPerCta = 64;    // query rows one CTA carries at most
+constexpr int kFp8TokenBytes = 656;
+
+// device status bits (sticky, in the first word of the workspace)
+constexpr int kStatusWaitTimeout = 1;
+
+struct DecodeParams {
+  const int32_t* block_table;
+  const int32_t* cache_seqlens;
+  const int32_t* tile_md;
+  const int32_t* num_splits;
+  __nv_bfloat16* out;     // [b, s_q, h_q, 512]
+  float* lse;             // [b, h_q, s_q]
+  float* o_part;          // [max_splits, R, 512]
+  float* lse_part;        // [max_splits, R]
+  int* status;
+  const uint8_t* kv_raw;  // FP8 cache base (656-byte tokens); unused for bf16
+  int max_blocks;
+  int batch;
+  int num_sm_parts;
+  int s_q;
+  int h_q;
+  int rows;               // R = s_q * h_q / h_kv
+  int row_groups;         // G = ceil(R / rows per CTA)
+  int causal;
+  float scale_log2;       // softmax_scale * log2(e)
+};
+
+struct CombineParams {
+  const int32_t* num_splits;
+  const float* o_part;
+  const float* lse_part;
+  __nv_bfloat16* out;
+  float* lse;
+  int batch;
+  int s_q;
+  int h_q;
+  int rows;
+};
+
+inline int row_groups_for(int rows) { return rows <= kRowsPerCta ? 1 : (rows + kRowsPerCta - 1) / kRowsPerCta; }
+
+// launchers (return cudaError_t as int)
+int launch_scheduler(const int32_t* cache_seqlens, int batch, int num_sm_parts, int32_t* tile_md,
+                     int32_t* num_splits, cudaStream_t stream);
+int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, int rows_per_cta,
+                       cudaStream_t stream);
+int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, cudaStream_t stream);
+int launch_combine(const CombineParams& p, cudaStream_t stream);
+
+}  // namespace mla

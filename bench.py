@@ -1,0 +1,313 @@
+"""Benchmark of MLA paged-KV decode on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: the tile scheduler
+(mla_get_metadata) and the split-KV decode with its combine (mla_decode_kvcache).
+The default workload is the memory-bound decode (batch 128, s_q 1, h_q 16, every
+cache length 8192, 64-token pages scattered by a seeded block table), whose KV cache
+(1.2 GB) is larger than the 126 MB L2, so no flush is needed between steps.
+
+value     KV bytes the step reads (exact token counts, 1152 B per bf16 token) plus q, out
+          and lse bytes, summed over all ranks, divided by the max-over-ranks device time
+          (CUDA events on the launching stream).
+e2e       the same metric when every step also copies its inputs (q, block_table,
+          cache_seqlens) from pinned host memory and reads back out and lse; the KV cache
+          is resident device state, as in serving.
+roofline  the decode call (main kernel + combine), algorithmic bytes per launch divided by
+          its mean CUDA-event duration, against the measured HBM copy bandwidth.
+cpu_baseline  the fp64 oracle timed on this host's cores on a bounded sample of requests.
+
+With N > 1 (torchrun), every rank runs its own batch of requests on its own GPU (requests
+are independent: weak scaling, no collective on the data path); the barrier and the
+max-over-ranks time use torch.distributed.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import threading
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _peaks():
+    try:
+        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for n, v in zip(names, s[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+def oracle_baseline(case, budget_s: float = 15.0):
+    """Time the fp64 oracle on a bounded prefix of the batch (about budget_s of host work)."""
+    import oracle
+    import mla_inputs as mi
+    t0 = time.perf_counter()
+    done = []
+    for b in range(case.batch):
+        oracle.mla_decode_reference(case, requests=[b])
+        done.append(b)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    sub = mi.DecodeCase(**{**case.__dict__, "cache_seqlens": case.cache_seqlens[done],
+                           "q_bits": case.q_bits[done], "block_table": case.block_table[done]})
+    units = mi.workload_units(sub)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    return {"seconds": dt, "requests": len(done), "units": units, "cores": int(cores)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mem_b128_h16_L8192")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    import mla_inputs as mi
+    w = mi.WORKLOADS[args.workload]
+    metric = "MLA paged-KV decode TFLOP/s and KV HBM GB/s; fraction of B200 roofline"
+    hbm_peak, tc_peak, tc_sustained, peak_kind = _peaks()
+
+    if args.impl == "reference":
+        # the reference arm is the fp64 oracle on host cores (rank 0 only)
+        if rank != 0:
+            return
+        case = mi.make_workload(args.workload, poison=False)
+        per_step = []
+        for _ in range(args.warmup + args.steps):
+            r = oracle_baseline(case, budget_s=max(1.0, args.cpu_budget / max(1, args.steps)))
+            per_step.append(r)
+        timed = per_step[args.warmup:]
+        byts = sum(r["units"]["bytes"] for r in timed)
+        secs = sum(r["seconds"] for r in timed)
+        value = byts / secs / 1e9
+        line = {"impl": "reference", "metric": metric, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(timed),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": args.workload, "batch": w.batch, "s_q": w.s_q,
+                                                 "h_q": w.h_q, "seqlens": w.seqlens, "kv": w.kv_format},
+                "cpu_baseline": {"value": value, "unit": "GB/s", "cores": timed[0]["cores"], "kind": "oracle",
+                                 "sample": f"first {timed[0]['requests']} of {w.batch} requests per step"},
+                "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import attention_mla_get_b200 as mla
+
+    def to_device(c, device):
+        qd = torch.from_numpy(c.q_bits.view(np.int16)).view(torch.bfloat16).to(device)
+        if c.kv_format == "bf16":
+            kvd = torch.from_numpy(c.kv.view(np.int16)).view(torch.bfloat16).reshape(
+                c.num_blocks, mi.PAGE, 1, mi.D_QK).to(device)
+        else:
+            kvd = torch.from_numpy(c.kv).to(device)
+        return qd, kvd, torch.from_numpy(c.block_table).to(device), torch.from_numpy(c.cache_seqlens).to(device)
+
+    # every rank owns its own requests (seed shifted by rank): independent problems
+    case = mi.make_workload(args.workload, poison=False)
+    if rank > 0:
+        case = mi.make_case(case.batch, case.s_q, case.h_q, case.cache_seqlens, causal=case.causal,
+                            kv_format=case.kv_format, seed=w.seed + 1000 * rank, poison=False)
+    units = mi.workload_units(case)
+    q, kv, bt, sl = to_device(case, dev)
+    R = case.rows
+    parts = mla.mla_num_sm_parts(R, 1, local)
+    ws = torch.zeros(mla.mla_workspace_size(case.batch, parts, R, 1), dtype=torch.uint8, device=dev)
+    out = torch.empty((case.batch, case.s_q, case.h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((case.batch, case.h_q, case.s_q), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        md, ns = mla.mla_get_metadata(sl, R, 1, num_sm_parts=parts)
+        mla.mla_decode_kvcache(q, kv, bt, sl, 512, md, ns, softmax_scale=case.softmax_scale, causal=case.causal,
+                               out=out, lse=lse, workspace=ws)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+
+    # ---- device-timed steps, with per-call events for the decode kernel's roofline ----
+    md0, ns0 = mla.mla_get_metadata(sl, R, 1, num_sm_parts=parts)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            md, ns = mla.mla_get_metadata(sl, R, 1, num_sm_parts=parts)
+            ev[i][0].record(stream)
+            mla.mla_decode_kvcache(q, kv, bt, sl, 512, md, ns, softmax_scale=case.softmax_scale,
+                                   causal=case.causal, out=out, lse=lse, workspace=ws)
+            ev[i][1].record(stream)
+        stop.record(stream)
+        barrier()
+    ms_total = max_over_ranks(start.elapsed_time(stop))
+    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    status = mla.mla_read_status(ws)
+
+    # ---- end to end through the C-ABI with host buffers ----
+    q_h = q.cpu().pin_memory()
+    bt_h = bt.cpu().pin_memory()
+    sl_h = sl.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    q_d, bt_d, sl_d = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(sl)
+    h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        bt_d.copy_(bt_h, non_blocking=True)
+        sl_d.copy_(sl_h, non_blocking=True)
+        md, ns = mla.mla_get_metadata(sl_d, R, 1, num_sm_parts=parts)
+        mla.mla_decode_kvcache(q_d, kv, bt_d, sl_d, 512, md, ns, softmax_scale=case.softmax_scale,
+                               causal=case.causal, out=out, lse=lse, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t2.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(s2.elapsed_time(t2))
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    total_bytes = units["bytes"] * world * args.steps
+    value = total_bytes / (ms_total * 1e-3) / 1e9
+    tflops = units["flops"] * world * args.steps / (ms_total * 1e-3) / 1e12
+    achieved = units["bytes"] / (decode_ms * 1e-3) / 1e9
+    roof_time = max(units["bytes"] / (hbm_peak * 1e9), units["flops"] / (tc_peak * 1e12))
+    line = {
+        "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": case.batch, "s_q": case.s_q, "h_q": case.h_q,
+                   "h_kv": 1, "d_qk": 576, "d_v": 512, "page": 64, "seqlens": w.seqlens, "causal": case.causal,
+                   "kv": case.kv_format, "kv_bytes": units["kv_bytes"], "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world} (independent requests per GPU)"},
+        "tflops": tflops,
+        "roofline_fraction": roof_time / (ms_total / args.steps * 1e-3),
+        "roofline": {"bound": "hbm" if units["bytes"] / (hbm_peak * 1e9) >= units["flops"] / (tc_peak * 1e12)
+                     else "tensor",
+                     "kernel": "mla_decode_kvcache (split-KV main + combine)", "achieved": achieved,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": None,
+                     "peak_kind": peak_kind},
+        "e2e": {"value": units["bytes"] * world * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+        "device_status": status,
+    }
+    if not args.no_cpu_baseline:
+        r = oracle_baseline(case, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": r["units"]["bytes"] / r["seconds"] / 1e9, "unit": "GB/s",
+                                "cores": r["cores"], "kind": "oracle",
+                                "sample": f"first {r['requests']} of {case.batch} requests, fp64 numpy"}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,142 @@
+/*
+ * libmla -- Multi-head Latent Attention decode over a paged KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (FlashMLA pages: mha_fwd_kvcache_mla in the "flash_api.cpp" excerpt of the
+ * mmssai.com page; get_mla_metadata / flash_mla_with_kvcache in the usage examples of the
+ * kdjingpai.com, aiboss88.com and deepseekonline.chat pages; the FP8 token layout table
+ * and the newer is_fp8 argument on the wmrh.cn page):
+ *
+ *   q        [batch, s_q, h_q, 576]            bf16   query rows (512 latent + 64 RoPE dims)
+ *   kvcache  [num_blocks, 64, h_kv, 576]        bf16   paged latent cache, 64-token pages
+ *            or [num_blocks, 64, 656]           u8     FP8 tokens: 512 e4m3 codes, 4 fp32
+ *                                                      scales (one per 128 dims), 64 bf16 RoPE
+ *   block_table [batch, max_blocks]             int32  page j of request b is block_table[b][j]
+ *   cache_seqlens [batch]                       int32  tokens cached per request (L_b)
+ *
+ *   For request b, query position i and head h (h_kv = 1: every head reads the same cache):
+ *     s_j  = softmax_scale * <q[b,i,h,:], K_b[j,:]>       over all 576 dims, j < L_b,
+ *            and, if causal, j <= L_b - s_q + i          (the queries sit at the end of the cache)
+ *     O[b,i,h,:] = sum_j softmax(s)_j * K_b[j, 0:512]     (V = first 512 dims of the cached vector)
+ *     LSE[b,h,i] = log sum_j exp(s_j)                     (natural log; -inf if no key is visible)
+ *
+ *   out [batch, s_q, h_q, 512] bf16,  lse [batch, h_q, s_q] fp32.
+ *
+ * Conventions for every call
+ *   - All pointers are DEVICE pointers unless stated otherwise; the caller owns every buffer.
+ *   - The library allocates no device memory and never synchronises the stream; calls are
+ *     enqueued on `stream` (a cudaStream_t, NULL = legacy default stream) and return at once.
+ *   - Return value: MLA_OK (0) or a negative MLA_ERR_* code.  Argument errors are detected on
+ *     the host before anything is enqueued.  A CUDA launch failure returns MLA_ERR_CUDA.
+ *   - Values inside device arrays (seqlens, block_table) are trusted: out-of-range page ids are
+ *     not detected (the copy engine reads zeros for pages outside the cache).
+ *   - Supported shapes: h_kv = 1, d_v = 512, head dim 576, page size 64, 1 <= s_q * h_q <= 4096.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_OK 0
+#define MLA_ERR_NULL_POINTER (-1)     /* a required pointer is NULL */
+#define MLA_ERR_MISALIGNED (-2)       /* q, kvcache, out or workspace not 16-byte aligned; lse not 4-byte */
+#define MLA_ERR_BAD_DIM (-3)          /* d_v != 512 */
+#define MLA_ERR_BAD_HEADS (-4)        /* h_kv != 1, h_q < 1, or h_q % h_kv != 0 */
+#define MLA_ERR_BAD_KV_DTYPE (-5)     /* kv_dtype not MLA_KV_BF16 / MLA_KV_FP8 */
+#define MLA_ERR_WORKSPACE (-6)        /* workspace_bytes < mla_workspace_size(...) */
+#define MLA_ERR_BAD_SHAPE (-7)        /* batch < 1, s_q < 1, num_blocks < 1, max_blocks < 1,
+                                         rows out of range, or num_blocks * 64 >= 2^31 */
+#define MLA_ERR_BAD_PARTS (-8)        /* num_sm_parts < 1 (pass the same value to
+                                         mla_get_metadata and mla_decode_kvcache) */
+#define MLA_ERR_NO_DEVICE (-9)        /* device query failed */
+#define MLA_ERR_CUDA (-100)           /* a CUDA runtime / driver call failed */
+
+#define MLA_KV_BF16 0                 /* kvcache bf16 [num_blocks, 64, 1, 576] */
+#define MLA_KV_FP8 1                  /* kvcache u8   [num_blocks, 64, 656]    */
+
+/* Device status bits written into the workspace by the kernels (sticky until reset). */
+#define MLA_STATUS_WAIT_TIMEOUT 1     /* an internal pipeline wait ran past its bound (~1 s);
+                                         the outputs of that call are undefined */
+
+/*
+ * Number of scheduler parts ("SM parts") for a problem: the number of CTAs that share one
+ * chunk of pages is G = ceil(rows_per_kv_head / 64) (1 when rows <= 64), so
+ * num_sm_parts = max(1, SM count of `device` / (h_kv * G)).
+ *   rows_per_kv_head  s_q * h_q / h_kv
+ * Returns the count (>= 1) or a negative MLA_ERR_* code.
+ */
+MLA_API int mla_num_sm_parts(int rows_per_kv_head, int h_kv, int device);
+
+/*
+ * Tile-scheduler metadata (get_mla_metadata): splits every request's 128-token blocks into
+ * chunks and spreads them over num_sm_parts parts so that each part carries about the same
+ * cost (blocks + a fixed cost of 2 blocks per chunk).  Run once per decode step; the result
+ * is reused by every layer.
+ *   cache_seqlens  device int32 [batch]
+ *   tile_md        device int32 [num_sm_parts, 8] (written): per part
+ *                  {begin_b, begin_block, end_b, end_block, first_split, 0, 0, 0}
+ *   num_splits     device int32 [batch + 1] (written): prefix count of chunks per request
+ * Errors: MLA_ERR_NULL_POINTER, MLA_ERR_BAD_SHAPE (batch < 1), MLA_ERR_BAD_HEADS,
+ *         MLA_ERR_BAD_PARTS, MLA_ERR_CUDA.
+ */
+MLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int rows_per_kv_head, int h_kv, int32_t* tile_md,
+                     int num_sm_parts, int32_t* num_splits, void* stream);
+
+/*
+ * Bytes of device workspace mla_decode_kvcache needs: a 256-byte status header, then fp32
+ * partial LSE [batch + num_sm_parts, rows] and partial O [batch + num_sm_parts, rows, 512]
+ * for requests split over several parts.  Returns 0 for invalid arguments.
+ */
+MLA_API size_t mla_workspace_size(int batch, int num_sm_parts, int rows_per_kv_head, int h_kv);
+
+/*
+ * MLA decode (flash_mla_with_kvcache / mha_fwd_kvcache_mla): split-KV main kernel then the
+ * LSE combine, both enqueued on `stream`.
+ *   q              device bf16 [batch, s_q, h_q, 576], contiguous, 16-byte aligned
+ *   kvcache        device, see kv_dtype; contiguous, 16-byte aligned
+ *   num_blocks     physical pages in kvcache
+ *   block_table    device int32 [batch, max_blocks], row-major
+ *   cache_seqlens  device int32 [batch]
+ *   h_kv           must be 1;  d_v must be 512
+ *   tile_md, num_splits   from mla_get_metadata with the same cache_seqlens and num_sm_parts
+ *   softmax_scale  multiplies q.k (e.g. 576^-0.5)
+ *   causal         0 / 1
+ *   kv_dtype       MLA_KV_BF16 or MLA_KV_FP8
+ *   out            device bf16 [batch, s_q, h_q, 512] (written)
+ *   lse            device fp32 [batch, h_q, s_q] (written)
+ *   workspace      device scratch of >= mla_workspace_size(batch, num_sm_parts, s_q*h_q, h_kv) bytes,
+ *                  16-byte aligned; its first word is the device status (MLA_STATUS_*)
+ */
+MLA_API int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, const int32_t* block_table,
+                       int max_blocks, const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                       int d_v, const int32_t* tile_md, int num_sm_parts, const int32_t* num_splits,
+                       float softmax_scale, int causal, int kv_dtype, void* out, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
+ * Reads the device status word of a workspace into *status (host pointer).  This call
+ * synchronises `stream`.  reset != 0 clears the word afterwards (enqueued on `stream`).
+ */
+MLA_API int mla_read_status(void* workspace, int reset, int* status, void* stream);
+
+/* Static description of an MLA_* code. Never NULL. */
+MLA_API const char* mla_strerror(int code);
+
+/* Library version, e.g. "0.1.0". */
+MLA_API const char* mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,158 @@
+"""GPU parity of the CUDA path (through the C-ABI) against the fp64 oracle.
+
+Tolerances: bf16 cache |dO| <= 5e-3 + 1e-2 |O_ref| element-wise, |dLSE| <= 1e-3;
+FP8 cache |dO| <= 2e-2 + 2e-2 |O_ref|.  The scheduler metadata must be bit-exact to the
+oracle's scheduler rule.  Sizes span several 128-token steps and ragged page tails; the
+full-size workloads are checked on sampled requests that the oracle computes one by one.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import mla_inputs as mi
+import oracle
+from tests._helpers import compare, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    import attention_mla_get_b200  # noqa: F401  (fails loudly if libmla.so is missing)
+    yield
+
+
+# ----------------------------------------------------------------------------- scheduler
+@pytest.mark.parametrize("seed", range(6))
+def test_scheduler_bit_exact(seed):
+    import attention_mla_get_b200 as mla
+    rng = np.random.default_rng(100 + seed)
+    B = int(rng.integers(1, 300))
+    sl = rng.integers(0, 20000, size=B).astype(np.int32)
+    sl[rng.random(B) < 0.1] = 0
+    for parts in (1, 7, 37, 74, 148, 400):
+        md, ns = mla.mla_get_metadata(torch.from_numpy(sl).cuda(), 16, 1, num_sm_parts=parts)
+        md_ref, ns_ref = oracle.schedule(sl, parts)
+        assert np.array_equal(md.cpu().numpy(), md_ref), parts
+        assert np.array_equal(ns.cpu().numpy(), ns_ref), parts
+
+
+def test_num_sm_parts_matches_rule():
+    import attention_mla_get_b200 as mla
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for rows in (1, 16, 32, 64, 65, 128, 256, 300):
+        assert mla.mla_num_sm_parts(rows, 1) == oracle.num_sm_parts_for(rows, 1, sms)
+
+
+# ----------------------------------------------------------------------------- parity
+CASES = [
+    # (name, batch, s_q, h_q, seqlens, causal)
+    ("r16_ragged", 4, 1, 16, [1, 200, 1000, 4097], False),
+    ("r16_short", 3, 1, 16, [63, 64, 65], False),
+    ("r8_pad_rows", 2, 1, 8, [300, 77], False),
+    ("r32", 3, 1, 32, [129, 640, 2049], False),
+    ("r32_causal_sq2", 3, 2, 16, [2, 130, 1000], True),
+    ("r64", 2, 1, 64, [500, 1537], False),
+    ("r128", 3, 1, 128, [64, 333, 2000], False),
+    ("r256_causal", 3, 2, 128, [2, 129, 1500], True),
+    ("r48_pad_groups", 2, 1, 48, [257, 1], False),
+    ("r96_two_groups", 2, 1, 96, [700, 128], False),
+]
+
+
+@pytest.mark.parametrize("name,batch,s_q,h_q,seqlens,causal", CASES, ids=[c[0] for c in CASES])
+@pytest.mark.parametrize("parts", [None, 1, 7])
+def test_parity_small(name, batch, s_q, h_q, seqlens, causal, parts):
+    case = mi.make_case(batch, s_q, h_q, seqlens, causal=causal, seed=zlib.crc32(name.encode()) % 1000, spare_blocks=2)
+    O_ref, L_ref = oracle.mla_decode_reference(case)
+    out, lse, status, _ = run_gpu(case, num_sm_parts=parts)
+    assert status == 0
+    compare(case, out, lse, O_ref, L_ref)
+
+
+def test_tiny_workload_exact_config():
+    case = mi.make_workload("tiny_b2_h16")
+    O_ref, L_ref = oracle.mla_decode_reference(case)
+    out, lse, status, _ = run_gpu(case)
+    assert status == 0
+    compare(case, out, lse, O_ref, L_ref)
+
+
+def test_zero_length_and_fully_masked_rows():
+    # request 1 has no cached token; request 0 (causal, L=1, s_q=3) has rows that see nothing
+    case = mi.make_case(3, 3, 16, [1, 0, 200], causal=True, seed=21)
+    O_ref, L_ref = oracle.mla_decode_reference(case)
+    out, lse, status, _ = run_gpu(case)
+    assert status == 0
+    compare(case, out, lse, O_ref, L_ref)
+
+
+def test_block_table_permutation_is_bit_invariant():
+    case = mi.make_case(3, 1, 16, [300, 1000, 77], seed=22)
+    out1, lse1, _, _ = run_gpu(case)
+    rng = np.random.default_rng(5)
+    perm = rng.permutation(case.num_blocks)
+    kv2 = np.empty_like(case.kv)
+    kv2[perm] = case.kv
+    bt2 = case.block_table.copy()
+    bt2[bt2 >= 0] = perm[bt2[bt2 >= 0]]
+    case2 = mi.DecodeCase(**{**case.__dict__, "kv": kv2, "block_table": bt2})
+    out2, lse2, _, _ = run_gpu(case2)
+    assert np.array_equal(out1, out2) and np.array_equal(lse1, lse2)
+
+
+def test_nan_in_unreadable_slots_does_not_leak():
+    clean = mi.make_case(3, 2, 16, [70, 130, 1], causal=True, seed=23, poison=False, spare_blocks=4)
+    dirty = mi.make_case(3, 2, 16, [70, 130, 1], causal=True, seed=23, poison=True, spare_blocks=4)
+    o1, l1, _, _ = run_gpu(clean)
+    o2, l2, _, _ = run_gpu(dirty)
+    assert np.isfinite(o2).all()
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_split_count_invariance():
+    case = mi.make_case(2, 1, 128, [5000, 3000], seed=24)
+    O_ref, L_ref = oracle.mla_decode_reference(case)
+    results = []
+    for parts in (1, 3, 74):
+        out, lse, status, _ = run_gpu(case, num_sm_parts=parts)
+        assert status == 0
+        compare(case, out, lse, O_ref, L_ref)
+        results.append((out, lse))
+    for out, lse in results[1:]:
+        assert np.abs(out - results[0][0]).max() <= 1e-2
+        assert np.abs(lse - results[0][1]).max() <= 1e-4
+
+
+def test_flashmla_style_aliases():
+    import attention_mla_get_b200 as mla
+    case = mi.make_case(2, 1, 16, [100, 500], seed=25)
+    q, kv, bt, sl = to_device(case)
+    md, ns = mla.get_mla_metadata(sl, case.s_q * case.h_q // 1, 1)
+    out, lse = mla.flash_mla_with_kvcache(q, kv, bt, sl, 512, md, ns, causal=False)
+    O_ref, L_ref = oracle.mla_decode_reference(case)
+    compare(case, out.float().cpu().numpy(), lse.cpu().numpy(), O_ref, L_ref)
+
+
+# ------------------------------------------------------------------ full-size workloads
+FULL = ["mem_b128_h16_L8192", "varlen_b128_h128", "causal_b64_sq2_h128"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload_sampled(name):
+    case = mi.make_workload(name)
+    out, lse, status, (md, ns) = run_gpu(case)
+    assert status == 0
+    assert np.isfinite(out).all()
+    ns_h = ns.cpu().numpy()
+    md_ref, ns_ref = oracle.schedule(case.cache_seqlens, md.shape[0])
+    assert np.array_equal(md.cpu().numpy(), md_ref) and np.array_equal(ns_h, ns_ref)
+    # sample: the first and last request, the longest, and requests split over several parts
+    splits = np.diff(ns_h)
+    multi = [int(i) for i in np.nonzero(splits > 1)[0][:2]]
+    sample = sorted({0, case.batch - 1, int(np.argmax(case.cache_seqlens)), *multi})
+    O_ref, L_ref = oracle.mla_decode_reference(case, requests=sample)
+    compare(case, out, lse, O_ref, L_ref, requests=sample)
