@@ -128,7 +128,7 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   const int rg = rows_per_cta_for(rows);
 
   // q as a 3-D tensor {576 dims, rows, batch}; one box = 64 dims x rg rows of one request
-  CUtensorMap tm_q, tm_kv;
+  CUtensorMap tm_q, tm_kv, tm_scale, tm_rope;
   {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(rows),
                           static_cast<cuuint64_t>(batch)};
@@ -151,14 +151,21 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MLA_ERR_CUDA;
   } else {
-    // FP8 tokens as 2-D bytes {656, num_blocks * 64}; one box = 656 bytes would exceed the
-    // 256-element box limit, so the kernel reads 4 boxes of 164 bytes... see mla_decode_fp8.cu
+    // FP8 tokens as a 2-D byte tensor {656 bytes, num_blocks * 64 tokens}, read three ways:
+    // 128-byte columns of e4m3 codes, the 16 scale bytes at byte 512, and the 128 RoPE bytes
+    // at byte 528 with the 128-byte swizzle the MMA operand layout uses.
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kFp8TokenBytes), static_cast<cuuint64_t>(num_blocks) * kPage};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kFp8TokenBytes)};
-    cuuint32_t box[2] = {128, 64};
     cuuint32_t estr[2] = {1, 1};
-    if (encode(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(kvcache), dims, strides, box, estr,
+    cuuint32_t box_codes[2] = {128, 64}, box_scale[2] = {16, 64};
+    if (encode(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(kvcache), dims, strides, box_codes, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        encode(&tm_scale, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(kvcache), dims, strides, box_scale,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        encode(&tm_rope, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(kvcache), dims, strides, box_codes,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MLA_ERR_CUDA;
   }
@@ -187,7 +194,7 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int e = kv_dtype == MLA_KV_BF16 ? mla::launch_decode_bf16(tm_q, tm_kv, p, rg, st)
-                                  : mla::launch_decode_fp8(tm_q, tm_kv, p, st);
+                                  : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
 
   mla::CombineParams cp{};

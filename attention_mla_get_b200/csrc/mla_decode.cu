@@ -1,4 +1,4 @@
-// Split-KV MLA decode main kernel for sm_100a (bf16 paged KV cache).
+// Split-KV MLA decode main kernel for sm_100a (bf16 or FP8 paged KV cache).
 //
 // Problem (FlashMLA pages: mha_fwd_kvcache_mla / run_mha_fwd_splitkv_mla<bf16, 576> in the
 // "flash_api.cpp" excerpt, mmssai.com page; 64-token pages addressed by block_table,
@@ -29,6 +29,13 @@
 //                     PV(t) in order.  One HBM read, one shared-memory fill per byte.
 //   RELOAD (RG >= 32): K(t+1) is multiplied while softmax(t) runs; V(t) is reloaded
 //                     (an L2 hit) after K(t+1) because the ring cannot hold both steps.
+//
+// FP8 cache (656-byte tokens: 512 e4m3 codes, 4 fp32 scales, 64 bf16 RoPE dims; wmrh.cn
+// page, "FP8 KV缓存内存效率" table): the producer TMA-loads raw code columns (128 dims x 64
+// tokens) and the per-token scales into a raw ring; a dequant warpgroup (warps 6-9) writes
+// code * scale as bf16 into the same swizzled slot ring the MMA reads, and TMA-loads the RoPE
+// dims straight into their slot with the 128-byte swizzle.  Tokens past the end of the request
+// are written as zeros, so no tail fix-up is needed.  Always the RELOAD schedule.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -42,8 +49,9 @@ namespace {
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units (P <= 2^8)
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int RG, bool RETAIN>
+template <int RG, bool RETAIN, bool FP8>
 struct Cfg {
+  static constexpr int kThreads = FP8 ? 320 : 192;
   static constexpr int kSlotBytes = 32768;   // 128 tokens x 128 dims bf16
   static constexpr int kAtomColBytes = 16384;// 128 tokens x 64 dims (one swizzle column)
   static constexpr int kPageBoxBytes = 8192; // 64 tokens x 64 dims: one TMA box
@@ -52,12 +60,17 @@ struct Cfg {
   static constexpr int kPRowBytes = RG * 2;  // one token row of P^T (MN-major, rows contiguous)
   static constexpr int kPBytes = 128 * kPRowBytes;
   static constexpr int kNumP = (RG == 64) ? 1 : 2;
-  static constexpr int kNumSlots = RETAIN ? 6 : (RG == 64 ? 4 : 5);
+  static constexpr int kNumSlots = FP8 ? (RG == 64 ? 3 : (RG == 32 ? 4 : 5)) : (RETAIN ? 6 : (RG == 64 ? 4 : 5));
+  static constexpr int kNumRaw = FP8 ? 2 : 0;   // raw e4m3 code columns, 128 tokens x 128 bytes
+  static constexpr int kRawBytes = 16384;
+  static constexpr int kScaleBytes = 2048;       // 128 tokens x 4 fp32 scales
   static constexpr int kTmemCols = RG == 16 ? 128 : (RG == 32 ? 256 : 512);
   static constexpr int kOffQ = 0;
   static constexpr int kOffP = kOffQ + kQBytes;
   static constexpr int kOffSlots = kOffP + kNumP * kPBytes;
-  static constexpr int kOffMisc = kOffSlots + kNumSlots * kSlotBytes;
+  static constexpr int kOffRaw = kOffSlots + kNumSlots * kSlotBytes;
+  static constexpr int kOffScale = kOffRaw + kNumRaw * kRawBytes;
+  static constexpr int kOffMisc = kOffScale + (FP8 ? 2 * kScaleBytes : 0);
   static constexpr int kMiscBytes = 3072;
   static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
   static constexpr uint32_t kPSwzMask = RG / 8 - 1;                // (row bytes / 16) - 1
@@ -69,6 +82,7 @@ struct Cfg {
   static constexpr int kNOut = RG == 64 ? 2 : 1;  // columns per lane after a warp reduce-scatter
   static constexpr int kSlotsPerStep = RETAIN ? 5 : 9;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(!(FP8 && RETAIN), "the FP8 path always reloads V");
   static_assert(kQBytes % 1024 == 0 && kPBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
 };
 
@@ -85,7 +99,11 @@ enum : int {
   kBarOFull = 22,
   kBarOEmpty = 23,
   kBarDrain = 24,
-  kNumBars = 25,
+  kBarRawFull = 25,     // [2]
+  kBarRawEmpty = 27,    // [2]
+  kBarScaleFull = 29,   // [2]
+  kBarScaleEmpty = 31,  // [2]
+  kNumBars = 33,
 };
 
 __device__ __forceinline__ int blocks_of(int L) { return L > 0 ? (L + kBlockTokens - 1) / kBlockTokens : 0; }
@@ -164,11 +182,23 @@ __device__ __forceinline__ int col_of(int lane, int i) {
   else return lane >> 1;
 }
 
-template <int RG, bool RETAIN>
-__global__ void __launch_bounds__(192, 1)
-    mla_decode_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                           const DecodeParams p) {
-  using C = Cfg<RG, RETAIN>;
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes, float scale) {
+  uint32_t h;
+  const unsigned short c = static_cast<unsigned short>(two_codes & 0xFFFFu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(c));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16x2(f.x * scale, f.y * scale);
+}
+
+// tm_kv is the bf16 cache (64x64 boxes) or, for FP8, the byte view of the cache with 128-byte
+// code boxes; tm_scale (16-byte boxes at byte 512) and tm_rope (128-byte swizzled boxes at byte
+// 528) are used by the FP8 path only.
+template <int RG, bool RETAIN, bool FP8>
+__global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
+    mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                      const __grid_constant__ CUtensorMap tm_scale, const __grid_constant__ CUtensorMap tm_rope,
+                      const DecodeParams p) {
+  using C = Cfg<RG, RETAIN, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -177,12 +207,15 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sSlots = sbase + C::kOffSlots;
   uint8_t* misc = smem + C::kOffMisc;
   const uint32_t sBars = smem_u32(misc);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + 256);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 260);
-  float* red = reinterpret_cast<float*>(misc + 512);        // [4][64]
-  float* m_sm = reinterpret_cast<float*>(misc + 1536);      // [64]
-  float* alpha_sm = reinterpret_cast<float*>(misc + 1792);  // [64]
-  float* inv_sm = reinterpret_cast<float*>(misc + 2048);    // [64]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + 512);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 516);
+  float* red = reinterpret_cast<float*>(misc + 1024);       // [4][64]
+  float* m_sm = reinterpret_cast<float*>(misc + 2048);      // [64]
+  float* alpha_sm = reinterpret_cast<float*>(misc + 2304);  // [64]
+  float* inv_sm = reinterpret_cast<float*>(misc + 2560);    // [64]
+  static_assert(kNumBars * 8 <= 512, "barrier area");
+  const uint32_t sRaw = sbase + C::kOffRaw;
+  const uint32_t sScale = sbase + C::kOffScale;
   auto bar = [&](int i) -> uint32_t { return sBars + 8u * static_cast<uint32_t>(i); };
 
   const int warp = threadIdx.x >> 5;
@@ -207,12 +240,22 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarOEmpty), 4);
     mbar_init(bar(kBarDrain), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarRawFull + i), 1);
+      mbar_init(bar(kBarRawEmpty + i), 1);
+      mbar_init(bar(kBarScaleFull + i), 1);
+      mbar_init(bar(kBarScaleEmpty + i), 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_kv);
+    if (FP8) {
+      tma_prefetch_desc(&tm_scale);
+      tma_prefetch_desc(&tm_rope);
+    }
   }
   if (warp == 5) {
     tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
@@ -231,7 +274,75 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 4) {
     // ================================ TMA producer ================================
-    if (lane == 0) {
+    if constexpr (FP8) if (lane == 0) {
+      // raw e4m3 code columns and per-token scales for the dequant warpgroup
+      const uint64_t pol_keep = policy_evict_last();
+      const uint64_t pol_v = p.row_groups > 1 ? pol_keep : policy_evict_first();
+      uint32_t gr = 0, us = 0;
+      int last_raw[2] = {-1, -1}, last_scale[2] = {-1, -1};
+      int q_fills = 0;
+      bool ok = true;
+      ChunkWalk walk(p, part);
+      int b, c0, c1, split;
+      auto fill_raw = [&](int grp, int pA, int pB, bool hasB, uint64_t pol) -> bool {
+        const int r = static_cast<int>(gr % C::kNumRaw);
+        const uint32_t use = gr / C::kNumRaw;
+        if (!mbar_wait(bar(kBarRawEmpty + r), (use & 1u) ^ 1u, wc)) return false;
+        mbar_arrive_expect_tx(bar(kBarRawFull + r), (hasB ? 2u : 1u) * 8192u);
+        const uint32_t dst = sRaw + static_cast<uint32_t>(r) * C::kRawBytes;
+        tma_load_2d(dst, &tm_kv, 128 * grp, pA * kPage, bar(kBarRawFull + r), pol);
+        if (hasB) tma_load_2d(dst + 8192, &tm_kv, 128 * grp, pB * kPage, bar(kBarRawFull + r), pol);
+        last_raw[r] = static_cast<int>(use);
+        ++gr;
+        return true;
+      };
+      auto fill_scale = [&](int pA, int pB, bool hasB) -> bool {
+        const int sb = static_cast<int>(us & 1u);
+        const uint32_t use = us >> 1;
+        if (!mbar_wait(bar(kBarScaleEmpty + sb), (use & 1u) ^ 1u, wc)) return false;
+        mbar_arrive_expect_tx(bar(kBarScaleFull + sb), (hasB ? 2u : 1u) * 1024u);
+        const uint32_t dst = sScale + static_cast<uint32_t>(sb) * C::kScaleBytes;
+        tma_load_2d(dst, &tm_scale, kDv, pA * kPage, bar(kBarScaleFull + sb), pol_keep);
+        if (hasB) tma_load_2d(dst + 1024, &tm_scale, kDv, pB * kPage, bar(kBarScaleFull + sb), pol_keep);
+        last_scale[sb] = static_cast<int>(use);
+        ++us;
+        return true;
+      };
+      while (ok && walk.next(p, b, c0, c1, split)) {
+        const int L = p.cache_seqlens[b];
+        const int npages = (L + kPage - 1) / kPage;
+        const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
+        if (!mbar_wait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(bar(kBarQFull), 9u * C::kQAtomBytes);
+        for (int a = 0; a < 9; ++a) tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, 64 * a, rg * RG, b, bar(kBarQFull));
+        ++q_fills;
+        int prevA = 0, prevB = 0;
+        bool prevHasB = false;
+        for (int t = 0; ok && t < c1 - c0; ++t) {
+          const int blk = c0 + t;
+          const int pA = bt[2 * blk];
+          const bool hasB = 2 * blk + 1 < npages;
+          const int pB = hasB ? bt[2 * blk + 1] : 0;
+          ok = fill_scale(pA, pB, hasB);
+          for (int grp = 0; ok && grp < 4; ++grp) ok = fill_raw(grp, pA, pB, hasB, pol_keep);
+          if (t > 0)
+            for (int grp = 0; ok && grp < 4; ++grp) ok = fill_raw(grp, prevA, prevB, prevHasB, pol_v);
+          prevA = pA;
+          prevB = pB;
+          prevHasB = hasB;
+        }
+        for (int grp = 0; ok && grp < 4; ++grp) ok = fill_raw(grp, prevA, prevB, prevHasB, pol_v);
+      }
+      if (*abort_flag) {
+        for (int r = 0; r < 2; ++r) {
+          if (last_raw[r] >= 0) mbar_wait_drain(bar(kBarRawFull + r), static_cast<uint32_t>(last_raw[r]) & 1u);
+          if (last_scale[r] >= 0)
+            mbar_wait_drain(bar(kBarScaleFull + r), static_cast<uint32_t>(last_scale[r]) & 1u);
+        }
+        if (q_fills > 0) mbar_wait_drain(bar(kBarQFull), static_cast<uint32_t>(q_fills - 1) & 1u);
+      }
+    }
+    if constexpr (!FP8) if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
       // dims < 512 are read again (V reload or the other row groups): keep them in L2
@@ -378,7 +489,7 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(bar(kBarDrain));
       mbar_wait_drain(bar(kBarDrain), 0);
     }
-  } else {
+  } else if (warp < 4) {
     // ============================ softmax + epilogue ==============================
     const int tid = threadIdx.x;  // 0..127: token lane of S^T, dim lane of O^T
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
@@ -494,7 +605,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           tmem_wait_st();
         }
-        if (t0 + kBlockTokens > L) {
+        if (!FP8 && t0 + kBlockTokens > L) {
           // tail step: zero the V rows of tokens past the end (their cache slots may hold NaN,
           // and 0 * NaN would poison O)
           for (int vs = 0; vs < 4; ++vs) {
@@ -571,6 +682,114 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
 
+  if constexpr (FP8) {
+    if (warp >= 6) {
+      // ============================ FP8 dequant warpgroup ==========================
+      // Produces the bf16 slots in the order the MMA consumes them: K(0), K(1), V(0),
+      // K(2), V(1), ..., V(n-1); slot 4 of K(t) is the RoPE part, copied by TMA.
+      const int dt = threadIdx.x - 192;  // token lane within a step
+      const uint64_t pol_rope = p.row_groups > 1 ? policy_evict_last() : policy_evict_first();
+      uint32_t gs = 0, gr = 0, us = 0;
+      int last_rope[6] = {-1, -1, -1, -1, -1, -1};
+      bool ok = true, aborted = false;
+      ChunkWalk walk(p, part);
+      int b, c0, c1, split;
+      // code * scale -> bf16 for 128 dims of this thread's token (zeros past the end)
+      auto dequant_slot = [&](int grp, uint32_t sbuf, int t0, int L) -> bool {
+        const uint32_t s = gs % C::kNumSlots;
+        const uint32_t r = gr % C::kNumRaw;
+        ok &= warp_wait(bar(kBarRawFull + r), (gr / C::kNumRaw) & 1u, wc, lane);
+        ok &= warp_wait(bar(kBarSlotEmpty + s), ((gs / C::kNumSlots) & 1u) ^ 1u, wc, lane);
+        const uint32_t dst = sSlots + s * C::kSlotBytes + static_cast<uint32_t>(dt) * 128u;
+        const uint32_t swz = static_cast<uint32_t>(dt & 7);
+        if (t0 + dt < L) {
+          float scale;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(scale)
+                       : "r"(sScale + sbuf * C::kScaleBytes + static_cast<uint32_t>(dt) * 16u + 4u * grp));
+          const uint32_t src = sRaw + r * C::kRawBytes + static_cast<uint32_t>(dt) * 128u;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t cc = static_cast<uint32_t>((c + dt) & 7);
+            uint32_t w0, w1, w2, w3;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(src + 16u * cc));
+            const uint32_t oc = 2u * cc;  // 16 codes -> output chunks oc, oc + 1 (8 dims each)
+            const uint32_t base = dst + (oc >> 3) * C::kAtomColBytes;
+            st_shared_v4(base + ((((oc & 7u) ^ swz)) << 4), e4m3x2_to_bf16x2(w0, scale),
+                         e4m3x2_to_bf16x2(w0 >> 16, scale), e4m3x2_to_bf16x2(w1, scale),
+                         e4m3x2_to_bf16x2(w1 >> 16, scale));
+            st_shared_v4(base + ((((oc + 1u) & 7u) ^ swz) << 4), e4m3x2_to_bf16x2(w2, scale),
+                         e4m3x2_to_bf16x2(w2 >> 16, scale), e4m3x2_to_bf16x2(w3, scale),
+                         e4m3x2_to_bf16x2(w3 >> 16, scale));
+          }
+        } else {
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) st_shared_v4(dst + a * C::kAtomColBytes + 16u * q, 0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        if (named_bar_any(2, 128, !ok)) return false;
+        if (dt == 0) {
+          mbar_arrive(bar(kBarSlotFull + s));
+          mbar_arrive(bar(kBarRawEmpty + r));
+        }
+        ++gs;
+        ++gr;
+        return true;
+      };
+      auto rope_slot = [&](int pA, int pB, bool hasB) {
+        const uint32_t s = gs % C::kNumSlots;
+        const uint32_t use = gs / C::kNumSlots;
+        if (dt == 0 && ok) {
+          ok = mbar_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc);
+          if (ok) {
+            mbar_arrive_expect_tx(bar(kBarSlotFull + s), (hasB ? 2u : 1u) * C::kPageBoxBytes);
+            const uint32_t dst = sSlots + s * C::kSlotBytes;
+            tma_load_2d(dst, &tm_rope, kDv + 16, pA * kPage, bar(kBarSlotFull + s), pol_rope);
+            if (hasB)
+              tma_load_2d(dst + C::kPageBoxBytes, &tm_rope, kDv + 16, pB * kPage, bar(kBarSlotFull + s), pol_rope);
+            last_rope[s] = static_cast<int>(use);
+          }
+        }
+        ++gs;
+      };
+      while (!aborted && walk.next(p, b, c0, c1, split)) {
+        const int L = p.cache_seqlens[b];
+        const int npages = (L + kPage - 1) / kPage;
+        const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
+        const int n = c1 - c0;
+        uint32_t su_prev = 0;
+        for (int t = 0; t < n && !aborted; ++t) {
+          const int blk = c0 + t;
+          const int t0 = blk * kBlockTokens;
+          const int pA = bt[2 * blk];
+          const bool hasB = 2 * blk + 1 < npages;
+          const int pB = hasB ? bt[2 * blk + 1] : 0;
+          const uint32_t su = us++;
+          ok &= warp_wait(bar(kBarScaleFull + (su & 1u)), (su >> 1) & 1u, wc, lane);
+          for (int grp = 0; grp < 4 && !aborted; ++grp)
+            aborted = !dequant_slot(grp, su & 1u, t0, L);
+          if (aborted) break;
+          rope_slot(pA, pB, hasB);
+          if (t > 0) {
+            for (int grp = 0; grp < 4 && !aborted; ++grp)
+              aborted = !dequant_slot(grp, su_prev & 1u, t0 - kBlockTokens, L);
+            if (!aborted && dt == 0) mbar_arrive(bar(kBarScaleEmpty + (su_prev & 1u)));
+          }
+          su_prev = su;
+        }
+        if (aborted) break;
+        const int tl = (c1 - 1) * kBlockTokens;
+        for (int grp = 0; grp < 4 && !aborted; ++grp) aborted = !dequant_slot(grp, su_prev & 1u, tl, L);
+        if (!aborted && dt == 0) mbar_arrive(bar(kBarScaleEmpty + (su_prev & 1u)));
+      }
+      if (dt == 0 && *abort_flag)
+        for (int s = 0; s < C::kNumSlots; ++s)
+          if (last_rope[s] >= 0) mbar_wait_drain(bar(kBarSlotFull + s), static_cast<uint32_t>(last_rope[s]) & 1u);
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 5) {
@@ -579,14 +798,15 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int RG, bool RETAIN>
-int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, cudaStream_t stream) {
-  using C = Cfg<RG, RETAIN>;
-  auto kern = mla_decode_bf16_kernel<RG, RETAIN>;
+template <int RG, bool RETAIN, bool FP8>
+int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_scale,
+                const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
+  using C = Cfg<RG, RETAIN, FP8>;
+  auto kern = mla_decode_kernel<RG, RETAIN, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid(p.num_sm_parts, p.row_groups, 1);
-  kern<<<grid, 192, C::kSmemBytes, stream>>>(tm_q, tm_kv, p);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, tm_scale, tm_rope, p);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -595,9 +815,19 @@ int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeP
 int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, int rows_per_cta,
                        cudaStream_t stream) {
   switch (rows_per_cta) {
-    case 16: return launch_impl<16, true>(tm_q, tm_kv, p, stream);
-    case 32: return launch_impl<32, false>(tm_q, tm_kv, p, stream);
-    case 64: return launch_impl<64, false>(tm_q, tm_kv, p, stream);
+    case 16: return launch_impl<16, true, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+    case 32: return launch_impl<32, false, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+    case 64: return launch_impl<64, false, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+    default: return static_cast<int>(cudaErrorInvalidValue);
+  }
+}
+
+int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
+                      const CUtensorMap& tm_rope, const DecodeParams& p, int rows_per_cta, cudaStream_t stream) {
+  switch (rows_per_cta) {
+    case 16: return launch_impl<16, false, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
+    case 32: return launch_impl<32, false, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
+    case 64: return launch_impl<64, false, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }
 }

@@ -62,7 +62,8 @@ int launch_scheduler(const int32_t* cache_seqlens, int batch, int num_sm_parts, 
                      int32_t* num_splits, cudaStream_t stream);
 int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, int rows_per_cta,
                        cudaStream_t stream);
-int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, cudaStream_t stream);
+int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
+                      const CUtensorMap& tm_rope, const DecodeParams& p, int rows_per_cta, cudaStream_t stream);
 int launch_combine(const CombineParams& p, cudaStream_t stream);
 
 }  // namespace mla

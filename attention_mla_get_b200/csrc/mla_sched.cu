@@ -3,75 +3,145 @@
 // excerpt on the mmssai.com page; the scheduler balances requests and blocks over the
 // SMs, wmrh.cn page "计算流水线设计").
 //
-// The rule is integer-only and runs in one thread: it is O(batch + num_sm_parts) work
-// done once per decode step and reused by every layer.  It is:
-//   n_b      = ceil(L_b / 128) blocks (0 for L_b <= 0)
-//   T        = sum over n_b > 0 of (n_b + F),  F = kFixedSplitCost
-//   payload  = ceil(T / P) + F
-//   each part p, with budget = payload, takes chunks k = min(n_b - blk, budget - F)
-//   while budget > F, paying F + k per chunk, the cursor (b, blk) moving forward
-//   (skipping requests with n_b = 0).
-//   row p = {begin_b, begin_blk, end_b, end_blk, first_split, 0, 0, 0}
-//   num_splits[b+1] = num_splits[b] + chunks of b; a chunk's split index is
-//   num_splits[b] + its ordinal within b.
+// The rule (integer only):
+//   n_b    = ceil(L_b / 128) blocks (0 for L_b <= 0)
+//   cost   requests with n_b > 0 laid end to end, F + n_b units each (F = kFixedSplitCost);
+//          C_b = start of request b, block j of request b sits at C_b + F + j, T = total
+//   q      = ceil(T / P); part p owns the positions [p*q, (p+1)*q)
+//   row p  = {begin_b, begin_blk, end_b, end_blk, first_split, 0, 0, 0} where begin / end are
+//            the first block at a position >= p*q / >= (p+1)*q; (batch, 0) when there is none
+//   chunks of b = (last owner part) - (first owner part) + 1 = floor((C_b+F+n_b-1)/q) - floor((C_b+F)/q) + 1
+//   num_splits = prefix sum of chunks; first_split = num_splits[begin_b] + p - floor((C_b+F)/q)
+// Every quantity is a closed form of prefix sums, so one CTA of 1024 threads computes the
+// metadata in a few microseconds: a scan of costs, a binary search per part, a scan of
+// chunk counts.
 #include "mla_internal.h"
 
 namespace mla {
 
-__device__ __forceinline__ int blocks_of(int L) { return L > 0 ? (L + kBlockTokens - 1) / kBlockTokens : 0; }
+namespace {
 
-__global__ void __launch_bounds__(32) mla_tile_scheduler_kernel(const int32_t* __restrict__ seqlens, int batch,
-                                                                int parts, int32_t* __restrict__ md,
-                                                                int32_t* __restrict__ num_splits) {
-  if (threadIdx.x != 0) return;
-  const int F = kFixedSplitCost;
-  long long T = 0;
-  for (int b = 0; b < batch; ++b) {
-    const int n = blocks_of(seqlens[b]);
-    num_splits[b + 1] = 0;  // chunk counts first, prefix sums after the walk
-    if (n > 0) T += n + F;
+constexpr int kSchedThreads = 1024;
+
+__device__ __forceinline__ long long blocks_of(int L) { return L > 0 ? (L + kBlockTokens - 1) / kBlockTokens : 0; }
+
+// Inclusive scan of v over the CTA; returns the thread's inclusive prefix, *total gets the sum.
+__device__ long long block_scan(long long v, long long* warp_tot, long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
   }
-  num_splits[0] = 0;
-  const long long payload = (T + parts - 1) / parts + F;
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    warp_tot[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const long long before = warp == 0 ? 0 : warp_tot[warp - 1];
+  const long long tot = warp_tot[31];
+  __syncthreads();
+  if (total) *total = tot;
+  return v + before;
+}
 
-  int b = 0;
-  while (b < batch && blocks_of(seqlens[b]) == 0) ++b;
-  int blk = 0;
-  for (int p = 0; p < parts; ++p) {
-    const int begin_b = b, begin_blk = blk;
-    const int first_ordinal = b < batch ? num_splits[b + 1] : 0;
-    long long budget = payload;
-    while (budget > F && b < batch) {
-      const int n = blocks_of(seqlens[b]);
-      const long long room = budget - F;
-      const int k = (n - blk) < room ? (n - blk) : static_cast<int>(room);
-      num_splits[b + 1] += 1;
-      budget -= F + k;
-      blk += k;
-      if (blk == n) {
-        ++b;
-        while (b < batch && blocks_of(seqlens[b]) == 0) ++b;
-        blk = 0;
-      }
+__global__ void __launch_bounds__(kSchedThreads)
+    mla_tile_scheduler_kernel(const int32_t* __restrict__ seqlens, int batch, int parts, int32_t* __restrict__ md,
+                              int32_t* __restrict__ ns) {
+  __shared__ long long warp_tot[32];
+  const long long F = kFixedSplitCost;
+  const int tid = threadIdx.x;
+
+  // pass 1: ns[b + 1] = C_{b+1} (inclusive prefix of costs), T
+  long long carry = 0;
+  for (int base = 0; base < batch; base += kSchedThreads) {
+    const int b = base + tid;
+    const long long n = b < batch ? blocks_of(seqlens[b]) : 0;
+    long long tile_total;
+    const long long incl = block_scan(n > 0 ? n + F : 0, warp_tot, &tile_total) + carry;
+    if (b < batch) ns[b + 1] = static_cast<int32_t>(incl);
+    carry += tile_total;
+  }
+  if (tid == 0) ns[0] = 0;
+  const long long T = carry;
+  const long long q = T > 0 ? (T + parts - 1) / parts : 1;
+  __syncthreads();
+
+  // pass 2: per part, the first block at a position >= x (binary search on C_{b+1})
+  auto find = [&](long long x, int& fb, int& fj) {
+    int lo = 0, hi = batch;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (static_cast<long long>(ns[mid + 1]) > x) hi = mid;
+      else lo = mid + 1;
+    }
+    fb = lo;
+    if (lo >= batch) {
+      fj = 0;
+      return;
+    }
+    const long long cb = lo == 0 ? 0 : ns[lo];
+    const long long j = x - (cb + F);
+    fj = j > 0 ? static_cast<int>(j) : 0;
+  };
+  for (int p = tid; p < parts; p += kSchedThreads) {
+    int bb, bj, eb, ej;
+    find(static_cast<long long>(p) * q, bb, bj);
+    find(static_cast<long long>(p + 1) * q, eb, ej);
+    int ordinal = 0;
+    if ((bb != eb || bj != ej) && bb < batch) {
+      const long long cb = bb == 0 ? 0 : ns[bb];
+      ordinal = static_cast<int>(p - (cb + F) / q);
     }
     int32_t* row = md + static_cast<long long>(p) * kMdInts;
-    row[0] = begin_b;
-    row[1] = begin_blk;
-    row[2] = b;
-    row[3] = blk;
-    row[4] = first_ordinal;  // made absolute below
+    row[0] = bb;
+    row[1] = bj;
+    row[2] = eb;
+    row[3] = ej;
+    row[4] = ordinal;  // made absolute in pass 4
     row[5] = row[6] = row[7] = 0;
   }
-  for (int i = 0; i < batch; ++i) num_splits[i + 1] += num_splits[i];
-  for (int p = 0; p < parts; ++p) {
+  __syncthreads();
+
+  // pass 3: ns = prefix sum of chunk counts (costs are scanned again instead of read back,
+  // because ns is overwritten here)
+  carry = 0;
+  long long chunk_carry = 0;
+  for (int base = 0; base < batch; base += kSchedThreads) {
+    const int b = base + tid;
+    const long long n = b < batch ? blocks_of(seqlens[b]) : 0;
+    long long tile_total;
+    const long long incl = block_scan(n > 0 ? n + F : 0, warp_tot, &tile_total) + carry;
+    const long long cb = incl - (n > 0 ? n + F : 0);
+    const long long chunks = n > 0 ? (cb + F + n - 1) / q - (cb + F) / q + 1 : 0;
+    long long chunk_total;
+    const long long cincl = block_scan(chunks, warp_tot, &chunk_total) + chunk_carry;
+    if (b < batch) ns[b + 1] = static_cast<int32_t>(cincl);
+    carry += tile_total;
+    chunk_carry += chunk_total;
+  }
+  __syncthreads();
+
+  // pass 4: absolute split index of each part's first chunk
+  for (int p = tid; p < parts; p += kSchedThreads) {
     int32_t* row = md + static_cast<long long>(p) * kMdInts;
-    row[4] += num_splits[row[0]];
+    row[4] += ns[row[0]];
   }
 }
 
+}  // namespace
+
 int launch_scheduler(const int32_t* cache_seqlens, int batch, int num_sm_parts, int32_t* tile_md,
                      int32_t* num_splits, cudaStream_t stream) {
-  mla_tile_scheduler_kernel<<<1, 32, 0, stream>>>(cache_seqlens, batch, num_sm_parts, tile_md, num_splits);
+  mla_tile_scheduler_kernel<<<1, kSchedThreads, 0, stream>>>(cache_seqlens, batch, num_sm_parts, tile_md,
+                                                             num_splits);
   return static_cast<int>(cudaGetLastError());
 }
 

@@ -46,33 +46,51 @@ def _peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples SM clock, power and clock-event reasons through NVML every 10 ms while the
+    timed region runs (nvidia-smi as a fallback)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown"}
 
-    def __init__(self, device_index: int):
-        self.dev = device_index
-        self.samples = []
+    def __init__(self, torch_device):
+        self.samples = []           # (t, sm_mhz, max_mhz, power_w, reason_bits)
         self._stop = threading.Event()
         self._t = None
+        self._h = None
+        self.window = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(torch_device)
+            bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nv = pynvml
+        except Exception:
+            self._h = None
+
+    def _read(self):
+        nv, h = self._nv, self._h
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        try:
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:
+            rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        return sm, mx, pw, rs
 
     def _run(self):
         while not self._stop.is_set():
             try:
-                out = subprocess.run(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                                     timeout=5).stdout.strip()
-                if out:
-                    self.samples.append([x.strip() for x in out.split(",")])
+                self.samples.append((time.perf_counter(), *self._read()))
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            self._stop.wait(0.01)
 
     def __enter__(self):
-        self._t = threading.Thread(target=self._run, daemon=True)
-        self._t.start()
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
         return self
 
     def __exit__(self, *a):
@@ -80,19 +98,22 @@ class ClockSampler:
         if self._t:
             self._t.join(timeout=10)
 
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        inside = [s for s in self.samples if self.window and self.window[0] <= s[0] <= self.window[1]]
+        use = inside if len(inside) >= 3 else self.samples
         reasons = set()
-        for s in self.samples:
-            for n, v in zip(names, s[5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(self.samples)}
+        for s in use:
+            for bit, name in self.REASONS.items():
+                if s[4] & bit:
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([s[1] for s in use])), "sm_max_mhz": float(max(s[2] for s in use)),
+                "power_w_max": float(max(s[3] for s in use)), "reasons": sorted(reasons),
+                "samples": len(use), "scope": "timed region" if use is inside else "warm-up and timed region"}
 
 
 def oracle_baseline(case, budget_s: float = 15.0):
@@ -118,15 +139,41 @@ def oracle_baseline(case, budget_s: float = 15.0):
     return {"seconds": dt, "requests": len(done), "units": units, "cores": int(cores)}
 
 
+def rank_case(workload: str, rank: int, batch=None):
+    """The batch of requests rank `rank` owns: the named workload's shapes and cache lengths,
+    with the random contents drawn from a seed shifted by the rank (independent problems)."""
+    import mla_inputs as mi
+    w = mi.WORKLOADS[workload]
+    case = mi.make_workload(workload, poison=False, batch=batch)
+    if rank > 0:
+        case = mi.make_case(case.batch, case.s_q, case.h_q, case.cache_seqlens, causal=case.causal,
+                            kv_format=case.kv_format, seed=w.seed + 1000 * rank, poison=False, name=workload)
+    return case
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="mem_b128_h16_L8192")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="run the first BATCH requests of the workload (profiling captures)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -181,10 +228,7 @@ def main():
         return qd, kvd, torch.from_numpy(c.block_table).to(device), torch.from_numpy(c.cache_seqlens).to(device)
 
     # every rank owns its own requests (seed shifted by rank): independent problems
-    case = mi.make_workload(args.workload, poison=False)
-    if rank > 0:
-        case = mi.make_case(case.batch, case.s_q, case.h_q, case.cache_seqlens, causal=case.causal,
-                            kv_format=case.kv_format, seed=w.seed + 1000 * rank, poison=False)
+    case = rank_case(args.workload, rank, args.batch)
     units = mi.workload_units(case)
     q, kv, bt, sl = to_device(case, dev)
     R = case.rows
@@ -205,13 +249,6 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         step()
     barrier()
@@ -221,7 +258,8 @@ def main():
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
+        t_wall0 = time.perf_counter()
         start.record(stream)
         for i in range(args.steps):
             md, ns = mla.mla_get_metadata(sl, R, 1, num_sm_parts=parts)
@@ -231,7 +269,8 @@ def main():
             ev[i][1].record(stream)
         stop.record(stream)
         barrier()
-    ms_total = max_over_ranks(start.elapsed_time(stop))
+        clk.mark(t_wall0, time.perf_counter())
+    ms_total = max_over_ranks(start.elapsed_time(stop), world, dev)
     decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     status = mla.mla_read_status(ws)
 
@@ -255,16 +294,18 @@ def main():
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    barrier()
-    s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    t2.record(stream)
-    barrier()
-    e2e_ms = max_over_ranks(s2.elapsed_time(t2))
+    e2e_ms = None
+    if not args.no_e2e:
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        t2.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(s2.elapsed_time(t2), world, dev)
 
     if rank != 0:
         if world > 1:
@@ -292,8 +333,9 @@ def main():
                      "kernel": "mla_decode_kvcache (split-KV main + combine)", "achieved": achieved,
                      "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": None,
                      "peak_kind": peak_kind},
-        "e2e": {"value": units["bytes"] * world * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": None if e2e_ms is None else {
+            "value": units["bytes"] * world * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
         "device_status": status,

@@ -8,27 +8,25 @@ spreads requests and blocks evenly over the SMs so that the load is balanced
 written once here and once in the CUDA scheduler kernel:
 
   unit          a block of 128 tokens (two 64-token pages); request b has
-                n_b = ceil(L_b / 128) blocks (0 when L_b = 0)
-  cost          every chunk costs F + (its blocks); F = FIXED_SPLIT_COST = 2 blocks
-  T             sum over requests with n_b > 0 of (n_b + F)
-  payload       ceil(T / num_sm_parts) + F
-  walk          parts p = 0 .. num_sm_parts-1 in order, with a cursor (b, blk) that
-                starts at the first request with n_b > 0.  Part p gets budget =
-                payload; while budget > F and requests remain it takes
-                k = min(n_b - blk, budget - F) blocks of request b as one chunk,
-                budget -= F + k, and moves the cursor (to the next request with
-                n_b > 0 when b is finished).
+                n_b = ceil(L_b / 128) blocks (0 when L_b <= 0)
+  cost line     requests with n_b > 0 are laid end to end, each taking F + n_b cost
+                units (F = FIXED_SPLIT_COST = 2: the cost of opening a chunk, then one
+                unit per block); C_b is where request b starts, block j of request b
+                sits at position C_b + F + j, and T is the total length
+  parts         q = ceil(T / num_sm_parts); part p owns the positions [p*q, (p+1)*q)
+  chunks        part p gets, for every request, the blocks whose positions it owns
+                (a contiguous run in (b, block) order)
   metadata row  {begin_b, begin_blk, end_b, end_blk, first_split, 0, 0, 0}: the part
-                covers the cursor range [begin, end) in (b, blk) order; a part with
-                no work has begin = end.
+                covers the cursor range [begin, end) in (b, block) order; a part with
+                no block has begin = end
   num_splits    num_splits[0] = 0, num_splits[b+1] = num_splits[b] + (chunks of b)
-  split index   of a chunk = num_splits[b] + its ordinal among b's chunks;
-                first_split = that index for the part's first chunk.
+  split index   of a chunk = num_splits[b] + (number of earlier parts holding blocks of b)
 
-Every block of every request lands in exactly one chunk: a part that ends inside a
-request has spent its whole payload, of which F pays for the extra chunk the
-next part opens, so each part covers at least ceil(T / num_sm_parts) of T.
-``schedule`` asserts it.
+Each part's cost (its blocks plus F per chunk) is at most q + F: the F units of every
+request that starts inside the part are on its interval, and only the first chunk of a
+part can be the continuation of a request started earlier.  Every block lands in
+exactly one chunk by construction.  Everything is a closed form of prefix sums, so the
+GPU kernel computes it in parallel.
 
 num_sm_parts: a CTA handles at most 64 query rows, so rows_per_kv_head rows need
 G = ceil(rows / 64) CTAs per chunk and num_sm_parts = max(1, sm_count // (h_kv * G)).
@@ -61,38 +59,54 @@ def schedule(cache_seqlens, num_sm_parts: int, fixed_cost: int = FIXED_SPLIT_COS
     B = len(L)
     P = int(num_sm_parts)
     assert P >= 1
+    F = int(fixed_cost)
     n = [_blocks(x) for x in L]
-    T = sum(nb + fixed_cost for nb in n if nb > 0)
-    payload = (T + P - 1) // P + fixed_cost
+    start = []                      # C_b
+    pos = 0
+    for nb in n:
+        start.append(pos)
+        if nb > 0:
+            pos += F + nb
+    T = pos
+    q = max(1, -(-T // P))
 
-    chunks_of = [0] * B
-    rows = []
+    # which part owns each block, by walking every block of every request
+    owner_runs = []                 # per request: list of (part, first_blk, end_blk)
+    for b in range(B):
+        runs = []
+        for j in range(n[b]):
+            part = (start[b] + F + j) // q
+            if runs and runs[-1][0] == part:
+                runs[-1][2] = j + 1
+            else:
+                runs.append([part, j, j + 1])
+        owner_runs.append(runs)
 
-    def skip_empty(b):
-        while b < B and n[b] == 0:
-            b += 1
-        return b
-
-    b, blk = skip_empty(0), 0
-    for _ in range(P):
-        begin_b, begin_blk = b, blk
-        first_ordinal = chunks_of[b] if b < B else 0
-        budget = payload
-        while budget > fixed_cost and b < B:
-            k = min(n[b] - blk, budget - fixed_cost)
-            chunks_of[b] += 1
-            budget -= fixed_cost + k
-            blk += k
-            if blk == n[b]:
-                b, blk = skip_empty(b + 1), 0
-        rows.append([begin_b, begin_blk, b, blk, first_ordinal])
-    assert b == B, "scheduler rule left work uncovered"
-
+    chunks_of = [len(r) for r in owner_runs]
     num_splits = np.zeros(B + 1, dtype=np.int32)
     num_splits[1:] = np.cumsum(chunks_of)
+
     md = np.zeros((P, MD_INTS), dtype=np.int32)
-    for p, (bb, bk, eb, ek, ordn) in enumerate(rows):
-        md[p, :5] = [bb, bk, eb, ek, int(num_splits[bb]) + ordn]
+    for p in range(P):
+        begin, end = (B, 0), (B, 0)
+        found = False
+        for b in range(B):
+            for k, (part, s, e) in enumerate(owner_runs[b]):
+                if part == p and not found:
+                    begin = (b, s)
+                    first_split = int(num_splits[b]) + k
+                    found = True
+        # end: the first block (in (b, blk) order) owned by a later part
+        done = False
+        for b in range(B):
+            for part, s, e in owner_runs[b]:
+                if part > p and not done:
+                    end = (b, s)
+                    done = True
+        if not found:
+            begin = end
+            first_split = int(num_splits[end[0]]) if end[0] < B else int(num_splits[B])
+        md[p, :5] = [begin[0], begin[1], end[0], end[1], first_split]
     return md, num_splits
 
 

@@ -156,3 +156,46 @@ def test_full_workload_sampled(name):
     sample = sorted({0, case.batch - 1, int(np.argmax(case.cache_seqlens)), *multi})
     O_ref, L_ref = oracle.mla_decode_reference(case, requests=sample)
     compare(case, out, lse, O_ref, L_ref, requests=sample)
+
+
+# ------------------------------------------------------------------------ FP8 cache
+FP8_CASES = [
+    ("fp8_r16", 3, 1, 16, [1, 300, 2049], False),
+    ("fp8_r32", 2, 1, 32, [64, 777], False),
+    ("fp8_r64", 2, 1, 64, [129, 1000], False),
+    ("fp8_r128", 2, 1, 128, [130, 1000], False),
+    ("fp8_r256_causal", 2, 2, 128, [3, 700], True),
+]
+
+
+@pytest.mark.parametrize("name,batch,s_q,h_q,seqlens,causal", FP8_CASES, ids=[c[0] for c in FP8_CASES])
+@pytest.mark.parametrize("parts", [None, 3])
+def test_parity_fp8_small(name, batch, s_q, h_q, seqlens, causal, parts):
+    case = mi.make_case(batch, s_q, h_q, seqlens, causal=causal, kv_format="fp8",
+                        seed=zlib.crc32(name.encode()) % 1000, spare_blocks=2)
+    O_ref, L_ref = oracle.mla_decode_reference(case)
+    out, lse, status, _ = run_gpu(case, num_sm_parts=parts)
+    assert status == 0
+    compare(case, out, lse, O_ref, L_ref)
+
+
+def test_fp8_nan_in_unreadable_slots_does_not_leak():
+    clean = mi.make_case(2, 1, 128, [70, 129], kv_format="fp8", seed=31, poison=False, spare_blocks=3)
+    dirty = mi.make_case(2, 1, 128, [70, 129], kv_format="fp8", seed=31, poison=True, spare_blocks=3)
+    o1, l1, _, _ = run_gpu(clean)
+    o2, l2, _, _ = run_gpu(dirty)
+    assert np.isfinite(o2).all()
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+@pytest.mark.slow
+def test_full_fp8_workload_sampled():
+    case = mi.make_workload("fp8_b128_h128_L16384")
+    out, lse, status, (md, ns) = run_gpu(case)
+    assert status == 0
+    assert np.isfinite(out).all()
+    ns_h = ns.cpu().numpy()
+    multi = [int(i) for i in np.nonzero(np.diff(ns_h) > 1)[0][:2]]
+    sample = sorted({0, case.batch - 1, *multi})
+    O_ref, L_ref = oracle.mla_decode_reference(case, requests=sample)
+    compare(case, out, lse, O_ref, L_ref, requests=sample)

@@ -90,28 +90,14 @@ def test_num_sm_parts_rule():
     assert ts.num_sm_parts_for(256, 1, 2) == 1
 
 
-def test_planted_payload_without_fixed_cost_fails():
-    """Dropping the +F from the payload leaves work uncovered for some batch."""
-    orig = ts.schedule
-
-    def bad(seqlens, parts, fixed=ts.FIXED_SPLIT_COST):
-        L = [int(x) for x in seqlens]
-        n = [ts._blocks(x) for x in L]
-        T = sum(nb + fixed for nb in n if nb > 0)
-        payload = -(-T // parts)            # planted: no + fixed
-        b, blk, covered = 0, 0, 0
-        for _ in range(parts):
-            budget = payload
-            while budget > fixed and b < len(L):
-                if n[b] == 0:
-                    b += 1
-                    continue
-                k = min(n[b] - blk, budget - fixed)
-                budget -= fixed + k
-                blk += k
-                covered += k
-                if blk == n[b]:
-                    b, blk = b + 1, 0
-        return covered == sum(n)
-    assert orig is ts.schedule
-    assert not all(bad([8192] * 128, 148, 2) for _ in range(1))
+def test_planted_floor_division_is_caught():
+    """With q = floor(T / parts) instead of the ceiling, some block's owner would be a part
+    index >= num_sm_parts for the memory-bound shape, i.e. left uncovered."""
+    seqlens = [8192] * 128
+    F, P = ts.FIXED_SPLIT_COST, 148
+    n = [ts._blocks(L) for L in seqlens]
+    T = sum(x + F for x in n)
+    q_bad = T // P
+    last_pos = T - 1
+    assert last_pos // q_bad >= P                       # the planted rule loses blocks
+    assert last_pos // (-(-T // P)) < P                 # the rule as written does not
