@@ -3,7 +3,7 @@
 #include <cstdio>
 #include <cstring>
 
-#include "../../include/mla.h"
+#include "mla.h"
 #include "mla_internal.h"
 
 namespace {

@@ -60,7 +60,7 @@ struct Cfg {
   static constexpr int kPRowBytes = RG * 2;  // one token row of P^T (MN-major, rows contiguous)
   static constexpr int kPBytes = 128 * kPRowBytes;
   static constexpr int kNumP = (RG == 64) ? 1 : 2;
-  static constexpr int kNumSlots = FP8 ? (RG == 64 ? 3 : (RG == 32 ? 4 : 5)) : (RETAIN ? 6 : (RG == 64 ? 4 : 5));
+  static constexpr int kNumSlots = FP8 ? (RG == 64 ? 3 : (RG == 32 ? 4 : 5)) : (RG == 16 ? 6 : (RG == 64 ? 4 : 5));
   static constexpr int kNumRaw = FP8 ? 2 : 0;   // raw e4m3 code columns, 128 tokens x 128 bytes
   static constexpr int kRawBytes = 16384;
   static constexpr int kScaleBytes = 2048;       // 128 tokens x 4 fp32 scales
