@@ -181,7 +181,6 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   p.lse_part = reinterpret_cast<float*>(ws + wl.lse_off);
   p.o_part = reinterpret_cast<float*>(ws + wl.o_off);
   p.status = reinterpret_cast<int*>(ws);
-  p.kv_raw = static_cast<const uint8_t*>(kvcache);
   p.max_blocks = max_blocks;
   p.batch = batch;
   p.num_sm_parts = num_sm_parts;

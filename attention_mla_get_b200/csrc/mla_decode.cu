@@ -60,8 +60,8 @@ struct Cfg {
   static constexpr int kPRowBytes = RG * 2;  // one token row of P^T (MN-major, rows contiguous)
   static constexpr int kPBytes = 128 * kPRowBytes;
   static constexpr int kNumP = (RG == 64) ? 1 : 2;
-  static constexpr int kNumSlots = FP8 ? (RG == 64 ? 3 : (RG == 32 ? 4 : 5)) : (RG == 16 ? 6 : (RG == 64 ? 4 : 5));
-  static constexpr int kNumRaw = FP8 ? 2 : 0;   // raw e4m3 code columns, 128 tokens x 128 bytes
+  static constexpr int kNumSlots = FP8 ? (RG == 64 ? 2 : (RG == 32 ? 3 : 4)) : (RG == 16 ? 6 : (RG == 64 ? 4 : 5));
+  static constexpr int kNumRaw = FP8 ? 4 : 0;   // raw e4m3 code columns, 128 tokens x 128 bytes
   static constexpr int kRawBytes = 16384;
   static constexpr int kScaleBytes = 2048;       // 128 tokens x 4 fp32 scales
   static constexpr int kTmemCols = RG == 16 ? 128 : (RG == 32 ? 256 : 512);
@@ -99,11 +99,11 @@ enum : int {
   kBarOFull = 22,
   kBarOEmpty = 23,
   kBarDrain = 24,
-  kBarRawFull = 25,     // [2]
-  kBarRawEmpty = 27,    // [2]
-  kBarScaleFull = 29,   // [2]
-  kBarScaleEmpty = 31,  // [2]
-  kNumBars = 33,
+  kBarRawFull = 25,     // [4]
+  kBarRawEmpty = 29,    // [4]
+  kBarScaleFull = 33,   // [2]
+  kBarScaleEmpty = 35,  // [2]
+  kNumBars = 37,
 };
 
 __device__ __forceinline__ int blocks_of(int L) { return L > 0 ? (L + kBlockTokens - 1) / kBlockTokens : 0; }
@@ -240,9 +240,11 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarOEmpty), 4);
     mbar_init(bar(kBarDrain), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(bar(kBarRawFull + i), 1);
       mbar_init(bar(kBarRawEmpty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarScaleFull + i), 1);
       mbar_init(bar(kBarScaleEmpty + i), 1);
     }
@@ -279,7 +281,7 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
       const uint64_t pol_keep = policy_evict_last();
       const uint64_t pol_v = p.row_groups > 1 ? pol_keep : policy_evict_first();
       uint32_t gr = 0, us = 0;
-      int last_raw[2] = {-1, -1}, last_scale[2] = {-1, -1};
+      int last_raw[4] = {-1, -1, -1, -1}, last_scale[2] = {-1, -1};
       int q_fills = 0;
       bool ok = true;
       ChunkWalk walk(p, part);
@@ -334,11 +336,11 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
         for (int grp = 0; ok && grp < 4; ++grp) ok = fill_raw(grp, prevA, prevB, prevHasB, pol_v);
       }
       if (*abort_flag) {
-        for (int r = 0; r < 2; ++r) {
+        for (int r = 0; r < 4; ++r)
           if (last_raw[r] >= 0) mbar_wait_drain(bar(kBarRawFull + r), static_cast<uint32_t>(last_raw[r]) & 1u);
+        for (int r = 0; r < 2; ++r)
           if (last_scale[r] >= 0)
             mbar_wait_drain(bar(kBarScaleFull + r), static_cast<uint32_t>(last_scale[r]) & 1u);
-        }
         if (q_fills > 0) mbar_wait_drain(bar(kBarQFull), static_cast<uint32_t>(q_fills - 1) & 1u);
       }
     }

@@ -31,7 +31,6 @@ struct DecodeParams {
   float* o_part;          // [max_splits, R, 512]
   float* lse_part;        // [max_splits, R]
   int* status;
-  const uint8_t* kv_raw;  // FP8 cache base (656-byte tokens); unused for bf16
   int max_blocks;
   int batch;
   int num_sm_parts;
