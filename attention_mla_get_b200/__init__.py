@@ -40,7 +40,7 @@ KV_FP8 = 1
 MLA_ERRORS = {
     -1: "MLA_ERR_NULL_POINTER", -2: "MLA_ERR_MISALIGNED", -3: "MLA_ERR_BAD_DIM", -4: "MLA_ERR_BAD_HEADS",
     -5: "MLA_ERR_BAD_KV_DTYPE", -6: "MLA_ERR_WORKSPACE", -7: "MLA_ERR_BAD_SHAPE", -8: "MLA_ERR_BAD_PARTS",
-    -9: "MLA_ERR_NO_DEVICE", -100: "MLA_ERR_CUDA",
+    -9: "MLA_ERR_NO_DEVICE", -10: "MLA_ERR_SCRATCH_LIMIT", -100: "MLA_ERR_CUDA",
 }
 
 
@@ -77,7 +77,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 
 EXPORTED = ("mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-            "mla_read_status", "mla_strerror", "mla_version")
+            "mla_decode_kvcache_noalloc", "mla_read_status", "mla_strerror", "mla_version")
 
 
 def mla_strerror(code: int) -> str:

@@ -69,6 +69,7 @@ const char* mla_strerror(int code) {
                                    "s_q*h_q <= 4096 and num_blocks*64 < 2^31";
     case MLA_ERR_BAD_PARTS: return "num_sm_parts must be >= 1";
     case MLA_ERR_NO_DEVICE: return "CUDA device query failed";
+    case MLA_ERR_SCRATCH_LIMIT: return "the problem's workspace exceeds the 16 MiB built-in scratch of the no-alloc call";
     case MLA_ERR_CUDA: return "a CUDA call failed";
     default: return "unknown libmla error code";
   }

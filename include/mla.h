@@ -59,6 +59,8 @@ extern "C" {
 #define MLA_ERR_BAD_PARTS (-8)        /* num_sm_parts < 1 (pass the same value to
                                          mla_get_metadata and mla_decode_kvcache) */
 #define MLA_ERR_NO_DEVICE (-9)        /* device query failed */
+#define MLA_ERR_SCRATCH_LIMIT (-10)   /* mla_decode_kvcache_noalloc: the problem needs more than
+                                         its 16 MiB built-in scratch array */
 #define MLA_ERR_CUDA (-100)           /* a CUDA runtime / driver call failed */
 
 #define MLA_KV_BF16 0                 /* kvcache bf16 [num_blocks, 64, 1, 576] */
@@ -122,6 +124,29 @@ MLA_API int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_b
                        int d_v, const int32_t* tile_md, int num_sm_parts, const int32_t* num_splits,
                        float softmax_scale, int causal, int kv_dtype, void* out, float* lse, void* workspace,
                        size_t workspace_bytes, void* stream);
+
+/*
+ * mla_decode_kvcache without a workspace argument, for callers that cannot allocate device
+ * memory when they run decode: engines that reserve all device memory at start-up and forbid
+ * later allocations, code running inside an allocator hook or driver callback where an
+ * allocation would re-enter the allocator, or plain C programs that link no allocator.
+ * (The FlashMLA pages have no counterpart of this call.)
+ *
+ * The workspace is a 16 MiB array inside this library, held by every GPU that loads it until
+ * the process exits.  Problems with mla_workspace_size(...) > 16 MiB return
+ * MLA_ERR_SCRATCH_LIMIT (e.g. batch 128 x 16 query rows fits, batch 128 x 128 rows does not).
+ * The first call on a device (with that device current) looks the array's address up once;
+ * make that first call before any stream capture.  All calls share the array and it keeps the
+ * last call's contents: the status word is cleared at the start of each call (an async memset
+ * on `stream`, no allocation), partial results are written before they are read.  Calls that
+ * overlap on the GPU (other streams or host threads) race on the array.  No cudaMalloc,
+ * cudaFree or allocating routine is called.  Other arguments and errors as mla_decode_kvcache.
+ */
+MLA_API int mla_decode_kvcache_noalloc(const void* q, const void* kvcache, int64_t num_blocks,
+                                       const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                                       int batch, int s_q, int h_q, int h_kv, int d_v, const int32_t* tile_md,
+                                       int num_sm_parts, const int32_t* num_splits, float softmax_scale, int causal,
+                                       int kv_dtype, void* out, float* lse, void* stream);
 
 /*
  * Reads the device status word of a workspace into *status (host pointer).  This call

@@ -38,7 +38,7 @@ def _declared():
 def test_every_declared_symbol_is_exported(lib):
     names = _declared()
     assert set(names) == {"mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-                          "mla_read_status", "mla_strerror", "mla_version"}
+                          "mla_decode_kvcache_noalloc", "mla_read_status", "mla_strerror", "mla_version"}
     so = os.path.join(ROOT, "attention_mla_get_b200", "libmla.so")
     nm = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True).stdout
     exported = set(re.findall(r" T (mla_\w+)", nm))
@@ -62,7 +62,7 @@ def test_built_for_sm100a():
 
 def test_strerror_and_version(lib):
     assert lib.mla_version() == b"0.1.0"
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -100, 12345):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10, -100, 12345):
         assert lib.mla_strerror(code)
 
 
