@@ -14,30 +14,32 @@
 // so O^T needs only 4*RG TMEM columns and the whole 512-dim output stays in TMEM.
 // A step covers 128 tokens (two 64-token pages).  Pages are TMA-loaded through the block
 // table in 64x64 boxes (the 9-boxes-per-page split on the wmrh.cn page, "内存访问优化策略")
-// into 32 KB ring slots (128 tokens x 128 dims, 128-byte swizzle).  The same slot is read
-// K-major by QK^T and MN-major (as V^T) by PV, so V is never transposed.
+// into 32 KB ring slots (128 tokens x 128 dims, 128-byte swizzle).  The same slot layout is
+// read K-major by QK^T and MN-major (as V^T) by PV, so V is never transposed.
 //
-// Roles (192 threads):  warps 0-3 online softmax + epilogue (thread = token lane of S^T,
-// then dim lane of O^T), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner.
+// Roles: warps 0-3 online softmax + epilogue (thread = token lane of S^T, then dim lane of
+// O^T), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner, warps 6-9 FP8 dequant.
 // Online softmax keeps a per-row running reference max (log2 units) and rescales O^T in
-// TMEM only when a block max exceeds it by more than kTau (the running-max-and-scale
-// idea of the wmrh.cn page, "跷跷板调度算法" paragraph); P^T is written to shared memory
-// as bf16, the row sums use the unrounded fp32 P.
+// TMEM only when a block max exceeds it by more than kTau (the running-max-and-scale idea
+// of the wmrh.cn page, "跷跷板调度算法" paragraph); P^T is written to shared memory as
+// bf16, the row sums use the unrounded fp32 P.
 //
-// Two load schedules:
-//   RELOAD (used for every shape): K(t+1) is multiplied while softmax(t) runs; V(t) is
-//                     reloaded (an L2 hit) after K(t+1) because the ring cannot hold both steps.
-//   RETAIN (kept as a template option): K(t) slots 0-3 are reused as V(t); QK(t) ->
-//                     softmax(t) -> PV(t) in order.  One shared-memory fill per byte, but the
-//                     tensor core idles during softmax; measured 9% slower on 16 query rows.
+// Issue order.  The ring of slots is filled and consumed in one fixed order per chunk of n
+// steps:  K(0) .. K(kLook),  then for t = 0 .. n-1:  V(t), K(t + kLook + 1).
+// K(t) is five slots (dims 0-127, ..., 384-511, and the 64 RoPE dims); V(t) is four slots
+// re-reading dims 0-511 of the same pages (an L2 hit).  QK(t) only needs K(t) and a free S^T
+// buffer, so it runs kLook steps ahead of PV(t), which waits for softmax(t).  Softmax
+// therefore always has kLook steps of MMA work to hide behind, the ring recycles at MMA
+// speed, and the tensor core never idles on the softmax (kLook + 1 S^T buffers in TMEM).
 //
 // FP8 cache (656-byte tokens: 512 e4m3 codes, 4 fp32 scales, 64 bf16 RoPE dims; wmrh.cn
 // page, "FP8 KV缓存内存效率" table): the producer TMA-loads raw code columns (128 dims x 64
-// tokens) and the per-token scales into a raw ring; a dequant warpgroup (warps 6-9) writes
-// code * scale as bf16 into the same swizzled slot ring the MMA reads, and TMA-loads the RoPE
-// dims straight into their slot with the 128-byte swizzle.  Tokens past the end of the request
-// are written as zeros, so no tail fix-up is needed.  Always the RELOAD schedule.
+// tokens) and the per-token scales into a raw ring; a dequant warpgroup writes code * scale as
+// bf16 into the same swizzled slot ring the MMA reads (same order as above), and TMA-loads the
+// RoPE dims straight into their slot with the 128-byte swizzle.  Tokens past the end of the
+// request are written as zeros, so no tail fix-up is needed.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "mla_internal.h"
@@ -49,8 +51,11 @@ namespace {
 
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units (P <= 2^8)
 constexpr float kLn2 = 0.69314718055994530942f;
+constexpr int kLook = 1;           // QK runs this many steps ahead of PV (2 measured no faster)
+constexpr int kNumS = kLook + 1;   // S^T buffers in TMEM
+constexpr int kMaxSlots = 6;
 
-template <int RG, bool RETAIN, bool FP8>
+template <int RG, bool FP8>
 struct Cfg {
   static constexpr int kThreads = FP8 ? 320 : 192;
   static constexpr int kSlotBytes = 32768;   // 128 tokens x 128 dims bf16
@@ -61,17 +66,18 @@ struct Cfg {
   static constexpr int kPRowBytes = RG * 2;  // one token row of P^T (MN-major, rows contiguous)
   static constexpr int kPBytes = 128 * kPRowBytes;
   static constexpr int kNumP = (RG == 64) ? 1 : 2;
-  static constexpr int kNumSlots = FP8 ? (RG == 64 ? 3 : (RG == 32 ? 4 : 5)) : (RG == 16 ? 6 : (RG == 64 ? 4 : 5));
+  static constexpr int kNumSlots = FP8 ? (RG == 64 ? 3 : 4) : (RG == 16 ? 6 : (RG == 64 ? 4 : 5));
   static constexpr int kNumRaw = FP8 ? 2 : 0;   // raw e4m3 code columns, 128 tokens x 128 bytes
   static constexpr int kRawBytes = 16384;
   static constexpr int kScaleBytes = 2048;       // 128 tokens x 4 fp32 scales
+  static constexpr int kNumScale = FP8 ? kNumS : 0;
   static constexpr int kTmemCols = RG == 16 ? 128 : (RG == 32 ? 256 : 512);
   static constexpr int kOffQ = 0;
   static constexpr int kOffP = kOffQ + kQBytes;
   static constexpr int kOffSlots = kOffP + kNumP * kPBytes;
   static constexpr int kOffRaw = kOffSlots + kNumSlots * kSlotBytes;
   static constexpr int kOffScale = kOffRaw + kNumRaw * kRawBytes;
-  static constexpr int kOffMisc = kOffScale + (FP8 ? 2 * kScaleBytes : 0);
+  static constexpr int kOffMisc = kOffScale + kNumScale * kScaleBytes;
   static constexpr int kMiscBytes = 3072;
   static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
   static constexpr uint32_t kPSwzMask = RG / 8 - 1;                // (row bytes / 16) - 1
@@ -79,31 +85,31 @@ struct Cfg {
   static constexpr uint32_t kIdescQK = idesc_bf16(128, RG, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16(128, RG, true, true);
   static constexpr int kColO = 0;       // 4 blocks of RG columns: O^T dims 128j..128j+127
-  static constexpr int kColS = 4 * RG;  // 2 buffers of RG columns: S^T
+  static constexpr int kColS = 4 * RG;  // kNumS buffers of RG columns: S^T
   static constexpr int kNOut = RG == 64 ? 2 : 1;  // columns per lane after a warp reduce-scatter
-  static constexpr int kSlotsPerStep = RETAIN ? 5 : 9;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(!(FP8 && RETAIN), "the FP8 path always reloads V");
+  static_assert(kNumSlots <= kMaxSlots, "slot barriers");
+  static_assert(kColS + kNumS * RG <= kTmemCols, "TMEM budget");
   static_assert(kQBytes % 1024 == 0 && kPBytes % 1024 == 0, "swizzle atoms need 1024-byte alignment");
 };
 
 // barrier indices in the misc area
 enum : int {
-  kBarSlotFull = 0,    // [6]
-  kBarSlotEmpty = 6,   // [6]
-  kBarSFull = 12,      // [2]
-  kBarSEmpty = 14,     // [2]
-  kBarPFull = 16,      // [2]
-  kBarPEmpty = 18,     // [2]
-  kBarQFull = 20,
-  kBarQEmpty = 21,
-  kBarOFull = 22,
-  kBarOEmpty = 23,
-  kBarDrain = 24,
-  kBarRawFull = 25,     // [4]
-  kBarRawEmpty = 29,    // [4]
-  kBarScaleFull = 33,   // [2]
-  kBarScaleEmpty = 35,  // [2]
+  kBarSlotFull = 0,     // [kMaxSlots]
+  kBarSlotEmpty = 6,    // [kMaxSlots]
+  kBarSFull = 12,       // [kNumS]
+  kBarSEmpty = 15,      // [kNumS]
+  kBarPFull = 18,       // [2]
+  kBarPEmpty = 20,      // [2]
+  kBarQFull = 22,
+  kBarQEmpty = 23,
+  kBarOFull = 24,
+  kBarOEmpty = 25,
+  kBarDrain = 26,
+  kBarRawFull = 27,     // [2]
+  kBarRawEmpty = 29,    // [2]
+  kBarScaleFull = 31,   // [kNumS]
+  kBarScaleEmpty = 34,  // [kNumS]
   kNumBars = 37,
 };
 
@@ -136,6 +142,31 @@ struct ChunkWalk {
     return false;
   }
 };
+
+// The fixed fill / consume order of one chunk of n steps: K(0) .. K(kLook), then V(t),
+// K(t + kLook + 1) for t = 0 .. n-1.  Entry e of the order is (is_v, step).
+__device__ __forceinline__ int order_len(int n) { return 2 * n; }
+__device__ __forceinline__ void order_at(int e, int n, bool& is_v, int& step) {
+  const int head = min(kLook + 1, n);
+  if (e < head) {
+    is_v = false;
+    step = e;
+    return;
+  }
+  const int r = e - head;           // alternating V(t), K(t + kLook + 1) while K steps remain
+  const int tail_k = n - head;      // K steps after the head
+  if (r < 2 * tail_k) {
+    is_v = (r & 1) == 0;
+    step = is_v ? (r >> 1) : (r >> 1) + head;
+  } else {
+    is_v = true;
+    step = tail_k + (r - 2 * tail_k);
+  }
+}
+// Slot fills of the chunk that precede V(t) slot 0 (each K step is 5 slots, each V step 4).
+__device__ __forceinline__ uint32_t slots_before_v(int t, int n) {
+  return 5u * static_cast<uint32_t>(min(t + kLook + 1, n)) + 4u * static_cast<uint32_t>(t);
+}
 
 // Drain wait used only after an abort: bounded, does not look at the abort flag.
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
@@ -191,21 +222,36 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes, float s
   return pack_bf16x2(f.x * scale, f.y * scale);
 }
 
+// Pages of step `st` of a request: page A always exists, page B only if the request has it.
+struct StepPages {
+  int a, b;
+  bool has_b;
+};
+__device__ __forceinline__ StepPages step_pages(const int32_t* bt, int st, int npages) {
+  StepPages sp;
+  sp.a = bt[2 * st];
+  sp.has_b = 2 * st + 1 < npages;
+  sp.b = sp.has_b ? bt[2 * st + 1] : 0;
+  return sp;
+}
+
 // tm_kv is the bf16 cache (64x64 boxes) or, for FP8, the byte view of the cache with 128-byte
 // code boxes; tm_scale (16-byte boxes at byte 512) and tm_rope (128-byte swizzled boxes at byte
 // 528) are used by the FP8 path only.
-template <int RG, bool RETAIN, bool FP8>
-__global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
+template <int RG, bool FP8>
+__global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                       const __grid_constant__ CUtensorMap tm_scale, const __grid_constant__ CUtensorMap tm_rope,
                       const DecodeParams p) {
-  using C = Cfg<RG, RETAIN, FP8>;
+  using C = Cfg<RG, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + C::kOffQ;
   const uint32_t sP = sbase + C::kOffP;
   const uint32_t sSlots = sbase + C::kOffSlots;
+  const uint32_t sRaw = sbase + C::kOffRaw;
+  const uint32_t sScale = sbase + C::kOffScale;
   uint8_t* misc = smem + C::kOffMisc;
   const uint32_t sBars = smem_u32(misc);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + 512);
@@ -215,8 +261,6 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
   float* alpha_sm = reinterpret_cast<float*>(misc + 2304);  // [64]
   float* inv_sm = reinterpret_cast<float*>(misc + 2560);    // [64]
   static_assert(kNumBars * 8 <= 512, "barrier area");
-  const uint32_t sRaw = sbase + C::kOffRaw;
-  const uint32_t sScale = sbase + C::kOffScale;
   auto bar = [&](int i) -> uint32_t { return sBars + 8u * static_cast<uint32_t>(i); };
 
   const int warp = threadIdx.x >> 5;
@@ -226,29 +270,27 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
   const WaitCtl wc{abort_flag, p.status, kStatusWaitTimeout};
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 6; ++i) {
+    for (int i = 0; i < kMaxSlots; ++i) {
       mbar_init(bar(kBarSlotFull + i), 1);
       mbar_init(bar(kBarSlotEmpty + i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNumS; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarSEmpty + i), 4);
+      mbar_init(bar(kBarScaleFull + i), 1);
+      mbar_init(bar(kBarScaleEmpty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarPFull + i), 4);
       mbar_init(bar(kBarPEmpty + i), 1);
+      mbar_init(bar(kBarRawFull + i), 1);
+      mbar_init(bar(kBarRawEmpty + i), 1);
     }
     mbar_init(bar(kBarQFull), 1);
     mbar_init(bar(kBarQEmpty), 1);
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarOEmpty), 4);
     mbar_init(bar(kBarDrain), 1);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(bar(kBarRawFull + i), 1);
-      mbar_init(bar(kBarRawEmpty + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarScaleFull + i), 1);
-      mbar_init(bar(kBarScaleEmpty + i), 1);
-    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -277,36 +319,63 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
 
   if (warp == 4) {
     // ================================ TMA producer ================================
-    if constexpr (FP8) if (lane == 0) {
-      // raw e4m3 code columns and per-token scales for the dequant warpgroup
+    if (lane == 0) {
+      const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
-      const uint64_t pol_v = p.row_groups > 1 ? pol_keep : policy_evict_first();
-      uint32_t gr = 0, us = 0;
-      int last_raw[4] = {-1, -1, -1, -1}, last_scale[2] = {-1, -1};
+      // dims < 512 are read again (V reload, other row groups): keep them in L2 until then
+      const uint64_t pol_v = p.row_groups > 1 ? pol_keep : pol_stream;
+      uint32_t g = 0;   // bf16 slot fills issued
+      uint32_t gr = 0;  // FP8 raw fills issued
+      uint32_t us = 0;  // FP8 scale fills issued
+      int last_use[kMaxSlots];
+      for (int i = 0; i < kMaxSlots; ++i) last_use[i] = -1;
+      int last_raw[2] = {-1, -1}, last_scale[kNumS];
+      for (int i = 0; i < kNumS; ++i) last_scale[i] = -1;
       int q_fills = 0;
       bool ok = true;
       ChunkWalk walk(p, part);
       int b, c0, c1, split;
-      auto fill_raw = [&](int grp, int pA, int pB, bool hasB, uint64_t pol) -> bool {
-        const int r = static_cast<int>(gr % C::kNumRaw);
-        const uint32_t use = gr / C::kNumRaw;
+      // one bf16 slot: natoms 64-dim columns starting at dims0, for the step's two pages
+      auto fill = [&](int dims0, int natoms, const StepPages& sp, uint64_t pol) -> bool {
+        const int s = static_cast<int>(g % C::kNumSlots);
+        const uint32_t use = g / C::kNumSlots;
+        if (!mbar_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
+        mbar_arrive_expect_tx(bar(kBarSlotFull + s),
+                              static_cast<uint32_t>(natoms * (sp.has_b ? 2 : 1) * C::kPageBoxBytes));
+        const uint32_t dst = sSlots + static_cast<uint32_t>(s) * C::kSlotBytes;
+        for (int a = 0; a < natoms; ++a) {
+          tma_load_2d(dst + a * C::kAtomColBytes, &tm_kv, dims0 + 64 * a, sp.a * kPage, bar(kBarSlotFull + s), pol);
+          if (sp.has_b)
+            tma_load_2d(dst + a * C::kAtomColBytes + C::kPageBoxBytes, &tm_kv, dims0 + 64 * a, sp.b * kPage,
+                        bar(kBarSlotFull + s), pol);
+        }
+        last_use[s] = static_cast<int>(use);
+        ++g;
+        return true;
+      };
+      // FP8: one raw column of e4m3 codes (group grp = dims 128grp..128grp+127)
+      auto fill_raw = [&](int grp, const StepPages& sp, uint64_t pol) -> bool {
+        constexpr uint32_t kRaw = C::kNumRaw > 0 ? C::kNumRaw : 1;
+        const int r = static_cast<int>(gr % kRaw);
+        const uint32_t use = gr / kRaw;
         if (!mbar_wait(bar(kBarRawEmpty + r), (use & 1u) ^ 1u, wc)) return false;
-        mbar_arrive_expect_tx(bar(kBarRawFull + r), (hasB ? 2u : 1u) * 8192u);
+        mbar_arrive_expect_tx(bar(kBarRawFull + r), (sp.has_b ? 2u : 1u) * 8192u);
         const uint32_t dst = sRaw + static_cast<uint32_t>(r) * C::kRawBytes;
-        tma_load_2d(dst, &tm_kv, 128 * grp, pA * kPage, bar(kBarRawFull + r), pol);
-        if (hasB) tma_load_2d(dst + 8192, &tm_kv, 128 * grp, pB * kPage, bar(kBarRawFull + r), pol);
+        tma_load_2d(dst, &tm_kv, 128 * grp, sp.a * kPage, bar(kBarRawFull + r), pol);
+        if (sp.has_b) tma_load_2d(dst + 8192, &tm_kv, 128 * grp, sp.b * kPage, bar(kBarRawFull + r), pol);
         last_raw[r] = static_cast<int>(use);
         ++gr;
         return true;
       };
-      auto fill_scale = [&](int pA, int pB, bool hasB) -> bool {
-        const int sb = static_cast<int>(us & 1u);
-        const uint32_t use = us >> 1;
+      // FP8: the per-token scales of one step
+      auto fill_scale = [&](const StepPages& sp) -> bool {
+        const int sb = static_cast<int>(us % kNumS);
+        const uint32_t use = us / kNumS;
         if (!mbar_wait(bar(kBarScaleEmpty + sb), (use & 1u) ^ 1u, wc)) return false;
-        mbar_arrive_expect_tx(bar(kBarScaleFull + sb), (hasB ? 2u : 1u) * 1024u);
+        mbar_arrive_expect_tx(bar(kBarScaleFull + sb), (sp.has_b ? 2u : 1u) * 1024u);
         const uint32_t dst = sScale + static_cast<uint32_t>(sb) * C::kScaleBytes;
-        tma_load_2d(dst, &tm_scale, kDv, pA * kPage, bar(kBarScaleFull + sb), pol_keep);
-        if (hasB) tma_load_2d(dst + 1024, &tm_scale, kDv, pB * kPage, bar(kBarScaleFull + sb), pol_keep);
+        tma_load_2d(dst, &tm_scale, kDv, sp.a * kPage, bar(kBarScaleFull + sb), pol_keep);
+        if (sp.has_b) tma_load_2d(dst + 1024, &tm_scale, kDv, sp.b * kPage, bar(kBarScaleFull + sb), pol_keep);
         last_scale[sb] = static_cast<int>(use);
         ++us;
         return true;
@@ -319,120 +388,81 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
         mbar_arrive_expect_tx(bar(kBarQFull), 9u * C::kQAtomBytes);
         for (int a = 0; a < 9; ++a) tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, 64 * a, rg * RG, b, bar(kBarQFull));
         ++q_fills;
-        int prevA = 0, prevB = 0;
-        bool prevHasB = false;
-        for (int t = 0; ok && t < c1 - c0; ++t) {
-          const int blk = c0 + t;
-          const int pA = bt[2 * blk];
-          const bool hasB = 2 * blk + 1 < npages;
-          const int pB = hasB ? bt[2 * blk + 1] : 0;
-          ok = fill_scale(pA, pB, hasB);
-          for (int grp = 0; ok && grp < 4; ++grp) ok = fill_raw(grp, pA, pB, hasB, pol_keep);
-          if (t > 0)
-            for (int grp = 0; ok && grp < 4; ++grp) ok = fill_raw(grp, prevA, prevB, prevHasB, pol_v);
-          prevA = pA;
-          prevB = pB;
-          prevHasB = hasB;
+        const int n = c1 - c0;
+        for (int e = 0; ok && e < order_len(n); ++e) {
+          bool is_v;
+          int t;
+          order_at(e, n, is_v, t);
+          const StepPages sp = step_pages(bt, c0 + t, npages);
+          if constexpr (FP8) {
+            if (!is_v) ok = fill_scale(sp);
+            for (int grp = 0; ok && grp < 4; ++grp) ok = fill_raw(grp, sp, is_v ? pol_v : pol_keep);
+          } else {
+            for (int ks = 0; ok && ks < 4; ++ks) ok = fill(128 * ks, 2, sp, is_v ? pol_v : pol_keep);
+            if (ok && !is_v) ok = fill(kDv, 1, sp, pol_stream);
+          }
         }
-        for (int grp = 0; ok && grp < 4; ++grp) ok = fill_raw(grp, prevA, prevB, prevHasB, pol_v);
-      }
-      if (*abort_flag) {
-        for (int r = 0; r < 4; ++r)
-          if (last_raw[r] >= 0) mbar_wait_drain(bar(kBarRawFull + r), static_cast<uint32_t>(last_raw[r]) & 1u);
-        for (int r = 0; r < 2; ++r)
-          if (last_scale[r] >= 0)
-            mbar_wait_drain(bar(kBarScaleFull + r), static_cast<uint32_t>(last_scale[r]) & 1u);
-        if (q_fills > 0) mbar_wait_drain(bar(kBarQFull), static_cast<uint32_t>(q_fills - 1) & 1u);
-      }
-    }
-    if constexpr (!FP8) if (lane == 0) {
-      const uint64_t pol_stream = policy_evict_first();
-      const uint64_t pol_keep = policy_evict_last();
-      // dims < 512 are read again (V reload or the other row groups): keep them in L2
-      const uint64_t pol_k = (!RETAIN || p.row_groups > 1) ? pol_keep : pol_stream;
-      const uint64_t pol_v = p.row_groups > 1 ? pol_keep : pol_stream;
-      uint32_t g = 0;  // slot fills issued
-      int last_use[6] = {-1, -1, -1, -1, -1, -1};
-      int q_fills = 0;
-      bool ok = true;
-      ChunkWalk walk(p, part);
-      int b, c0, c1, split;
-      auto fill = [&](int dims0, int natoms, int pA, int pB, bool hasB, uint64_t pol) -> bool {
-        const int s = static_cast<int>(g % C::kNumSlots);
-        const uint32_t use = g / C::kNumSlots;
-        if (!mbar_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
-        const uint32_t bytes = static_cast<uint32_t>(natoms * (hasB ? 2 : 1) * C::kPageBoxBytes);
-        mbar_arrive_expect_tx(bar(kBarSlotFull + s), bytes);
-        const uint32_t dst = sSlots + static_cast<uint32_t>(s) * C::kSlotBytes;
-        for (int a = 0; a < natoms; ++a) {
-          tma_load_2d(dst + a * C::kAtomColBytes, &tm_kv, dims0 + 64 * a, pA * kPage, bar(kBarSlotFull + s), pol);
-          if (hasB)
-            tma_load_2d(dst + a * C::kAtomColBytes + C::kPageBoxBytes, &tm_kv, dims0 + 64 * a, pB * kPage,
-                        bar(kBarSlotFull + s), pol);
-        }
-        last_use[s] = static_cast<int>(use);
-        ++g;
-        return true;
-      };
-      while (ok && walk.next(p, b, c0, c1, split)) {
-        const int L = p.cache_seqlens[b];
-        const int npages = (L + kPage - 1) / kPage;
-        const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
-        if (!mbar_wait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(bar(kBarQFull), 9u * C::kQAtomBytes);
-        for (int a = 0; a < 9; ++a) tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, 64 * a, rg * RG, b, bar(kBarQFull));
-        ++q_fills;
-        int prevA = 0, prevB = 0;
-        bool prevHasB = false;
-        for (int t = 0; ok && t < c1 - c0; ++t) {
-          const int blk = c0 + t;
-          const int pA = bt[2 * blk];
-          const bool hasB = 2 * blk + 1 < npages;
-          const int pB = hasB ? bt[2 * blk + 1] : 0;
-          for (int ks = 0; ok && ks < 4; ++ks) ok = fill(128 * ks, 2, pA, pB, hasB, pol_k);
-          if (ok) ok = fill(512, 1, pA, pB, hasB, pol_stream);
-          if (!RETAIN && t > 0)
-            for (int vs = 0; ok && vs < 4; ++vs) ok = fill(128 * vs, 2, prevA, prevB, prevHasB, pol_v);
-          prevA = pA;
-          prevB = pB;
-          prevHasB = hasB;
-        }
-        if (!RETAIN)
-          for (int vs = 0; ok && vs < 4; ++vs) ok = fill(128 * vs, 2, prevA, prevB, prevHasB, pol_v);
       }
       if (*abort_flag) {
         // let every copy this warp started land before the CTA may exit
         for (int s = 0; s < C::kNumSlots; ++s)
           if (last_use[s] >= 0) mbar_wait_drain(bar(kBarSlotFull + s), static_cast<uint32_t>(last_use[s]) & 1u);
+        for (int r = 0; r < 2; ++r)
+          if (last_raw[r] >= 0) mbar_wait_drain(bar(kBarRawFull + r), static_cast<uint32_t>(last_raw[r]) & 1u);
+        for (int r = 0; r < kNumS; ++r)
+          if (last_scale[r] >= 0)
+            mbar_wait_drain(bar(kBarScaleFull + r), static_cast<uint32_t>(last_scale[r]) & 1u);
         if (q_fills > 0) mbar_wait_drain(bar(kBarQFull), static_cast<uint32_t>(q_fills - 1) & 1u);
       }
     }
   } else if (warp == 5) {
     // ================================ MMA issuer ==================================
     if (lane == 0) {
-      uint32_t g = 0;  // slot fills consumed
-      uint32_t u = 0;  // global step counter (S / P buffers)
+      uint32_t g = 0;   // slot fills consumed
+      uint32_t u = 0;   // steps whose QK was issued (S^T buffers)
+      uint32_t up = 0;  // steps whose PV was issued (P buffers)
       int chunk = 0;
       bool ok = true;
       ChunkWalk walk(p, part);
       int b, c0, c1, split;
-      uint32_t gK_prev = 0;
-      auto do_pv = [&](int t, uint32_t uu, uint32_t gK) -> bool {
-        const int pb = static_cast<int>(uu % C::kNumP);
-        if (!mbar_wait(bar(kBarPFull + pb), (uu / C::kNumP) & 1u, wc)) return false;
-        if (t == 0 && !mbar_wait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) return false;
+      auto next_slot = [&](uint32_t& s) -> bool {
+        s = g % C::kNumSlots;
+        if (!mbar_wait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) return false;
+        ++g;
+        tc_fence_after();
+        return true;
+      };
+      auto do_qk = [&]() -> bool {
+        const int sb = static_cast<int>(u % kNumS);
+        if (!mbar_wait(bar(kBarSEmpty + sb), ((u / kNumS) & 1u) ^ 1u, wc)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + C::kColS + sb * RG;
+        for (int ks = 0; ks < 5; ++ks) {
+          uint32_t s;
+          if (!next_slot(s)) return false;
+          const uint32_t kbase = sSlots + s * C::kSlotBytes;
+          const int nk = ks < 4 ? 8 : 4;
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint32_t a = kbase + (kk >> 2) * C::kAtomColBytes + (kk & 3) * 32;
+            const uint32_t bq = sQ + (2 * ks + (kk >> 2)) * C::kQAtomBytes + (kk & 3) * 32;
+            umma_bf16(d, smem_desc(a, 16, 1024, kSwizzle128), smem_desc(bq, 16, 1024, kSwizzle128), C::kIdescQK,
+                      (ks | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(bar(kBarSlotEmpty + s));
+        }
+        umma_commit(bar(kBarSFull + sb));
+        ++u;
+        return true;
+      };
+      auto do_pv = [&](bool first_of_chunk) -> bool {
+        const int pb = static_cast<int>(up % C::kNumP);
+        if (!mbar_wait(bar(kBarPFull + pb), (up / C::kNumP) & 1u, wc)) return false;
+        if (first_of_chunk && !mbar_wait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) return false;
         tc_fence_after();
         const uint32_t pbase = sP + static_cast<uint32_t>(pb) * C::kPBytes;
         for (int vs = 0; vs < 4; ++vs) {
           uint32_t s;
-          if (RETAIN) {
-            s = (gK + vs) % C::kNumSlots;
-          } else {
-            s = g % C::kNumSlots;
-            if (!mbar_wait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) return false;
-            ++g;
-          }
-          tc_fence_after();
+          if (!next_slot(s)) return false;
           const uint32_t d = tmem + C::kColO + vs * RG;
           const uint32_t vbase = sSlots + s * C::kSlotBytes;
 #pragma unroll
@@ -440,50 +470,28 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
             const uint64_t adesc = smem_desc(vbase + kt * 2048, C::kAtomColBytes, 1024, kSwizzle128);
             const uint64_t bdesc = smem_desc(pbase + kt * 16 * C::kPRowBytes, 16 * 8 * C::kPRowBytes,
                                              8 * C::kPRowBytes, C::kPLayout);
-            umma_bf16(d, adesc, bdesc, C::kIdescPV, (t == 0 && kt == 0) ? 0u : 1u);
+            umma_bf16(d, adesc, bdesc, C::kIdescPV, (first_of_chunk && kt == 0) ? 0u : 1u);
           }
           umma_commit(bar(kBarSlotEmpty + s));
         }
         umma_commit(bar(kBarPEmpty + pb));
+        ++up;
         return true;
       };
       while (ok && walk.next(p, b, c0, c1, split)) {
         const int n = c1 - c0;
         if (!mbar_wait(bar(kBarQFull), chunk & 1, wc)) break;
-        for (int t = 0; ok && t < n; ++t) {
-          const int sb = static_cast<int>(u & 1u);
-          if (!mbar_wait(bar(kBarSEmpty + sb), ((u >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem + C::kColS + sb * RG;
-          const uint32_t gK = g;
-          for (int ks = 0; ks < 5; ++ks) {
-            const uint32_t s = g % C::kNumSlots;
-            if (!mbar_wait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t kbase = sSlots + s * C::kSlotBytes;
-            const int nk = ks < 4 ? 8 : 4;
-            for (int kk = 0; kk < nk; ++kk) {
-              const uint32_t a = kbase + (kk >> 2) * C::kAtomColBytes + (kk & 3) * 32;
-              const uint32_t bq = sQ + (2 * ks + (kk >> 2)) * C::kQAtomBytes + (kk & 3) * 32;
-              umma_bf16(d, smem_desc(a, 16, 1024, kSwizzle128), smem_desc(bq, 16, 1024, kSwizzle128), C::kIdescQK,
-                        (ks | kk) != 0 ? 1u : 0u);
-            }
-            if (!RETAIN || ks == 4) umma_commit(bar(kBarSlotEmpty + s));
-            ++g;
+        for (int e = 0; ok && e < order_len(n); ++e) {
+          bool is_v;
+          int t;
+          order_at(e, n, is_v, t);
+          if (is_v) {
+            ok = do_pv(t == 0);
+          } else {
+            ok = do_qk();
+            if (ok && t == n - 1) umma_commit(bar(kBarQEmpty));
           }
-          if (!ok) break;
-          umma_commit(bar(kBarSFull + sb));
-          if (t == n - 1) umma_commit(bar(kBarQEmpty));
-          if (RETAIN) {
-            ok = do_pv(t, u, gK);
-          } else if (t > 0) {
-            ok = do_pv(t - 1, u - 1, gK_prev);
-          }
-          gK_prev = gK;
-          ++u;
         }
-        if (!ok) break;
-        if (!RETAIN) ok = do_pv(n - 1, u - 1, gK_prev);
         if (!ok) break;
         umma_commit(bar(kBarOFull));
         ++chunk;
@@ -517,8 +525,8 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
       for (int t = 0; t < n; ++t) {
         const int t0 = (c0 + t) * kBlockTokens;
         const int j = t0 + tid;
-        const int sb = static_cast<int>(u & 1u);
-        bool ok = warp_wait(bar(kBarSFull + sb), (u >> 1) & 1u, wc, lane);
+        const int sb = static_cast<int>(u % kNumS);
+        bool ok = warp_wait(bar(kBarSFull + sb), (u / kNumS) & 1u, wc, lane);
         float x[RG];
         tc_fence_after();
 #pragma unroll
@@ -590,8 +598,8 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
         }
         if (rescale) {
           // O^T *= alpha per row, after PV(u - 1) has finished
-          const uint32_t up = u - 1;
-          ok &= warp_wait(bar(kBarPEmpty + up % C::kNumP), (up / C::kNumP) & 1u, wc, lane);
+          const uint32_t uq = u - 1;
+          ok &= warp_wait(bar(kBarPEmpty + uq % C::kNumP), (uq / C::kNumP) & 1u, wc, lane);
           tc_fence_after();
 #pragma unroll
           for (int vs = 0; vs < 4; ++vs) {
@@ -612,8 +620,7 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
           // tail step: zero the V rows of tokens past the end (their cache slots may hold NaN,
           // and 0 * NaN would poison O)
           for (int vs = 0; vs < 4; ++vs) {
-            const uint32_t gv = RETAIN ? gchunk + 5u * t + vs
-                                       : gchunk + 5u * static_cast<uint32_t>(min(t + 2, n)) + 4u * t + vs;
+            const uint32_t gv = gchunk + slots_before_v(t, n) + vs;
             const uint32_t s = gv % C::kNumSlots;
             ok &= warp_wait(bar(kBarSlotFull + s), (gv / C::kNumSlots) & 1u, wc, lane);
             if (j >= L) {
@@ -680,7 +687,7 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarOEmpty));
-      gchunk += static_cast<uint32_t>(C::kSlotsPerStep * n);
+      gchunk += 9u * static_cast<uint32_t>(n);
       ++chunk;
     }
   }
@@ -688,12 +695,13 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
   if constexpr (FP8) {
     if (warp >= 6) {
       // ============================ FP8 dequant warpgroup ==========================
-      // Produces the bf16 slots in the order the MMA consumes them: K(0), K(1), V(0),
-      // K(2), V(1), ..., V(n-1); slot 4 of K(t) is the RoPE part, copied by TMA.
+      // Produces the bf16 slots in the order the MMA consumes them (see the file header); slot 4
+      // of K(t) is the RoPE part, copied by TMA.
       const int dt = threadIdx.x - 192;  // token lane within a step
       const uint64_t pol_rope = p.row_groups > 1 ? policy_evict_last() : policy_evict_first();
       uint32_t gs = 0, gr = 0, us = 0;
-      int last_rope[6] = {-1, -1, -1, -1, -1, -1};
+      int last_rope[kMaxSlots];
+      for (int i = 0; i < kMaxSlots; ++i) last_rope[i] = -1;
       bool ok = true, aborted = false;
       ChunkWalk walk(p, part);
       int b, c0, c1, split;
@@ -741,17 +749,17 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
         ++gr;
         return true;
       };
-      auto rope_slot = [&](int pA, int pB, bool hasB) {
+      auto rope_slot = [&](const StepPages& sp) {
         const uint32_t s = gs % C::kNumSlots;
         const uint32_t use = gs / C::kNumSlots;
         if (dt == 0 && ok) {
           ok = mbar_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc);
           if (ok) {
-            mbar_arrive_expect_tx(bar(kBarSlotFull + s), (hasB ? 2u : 1u) * C::kPageBoxBytes);
+            mbar_arrive_expect_tx(bar(kBarSlotFull + s), (sp.has_b ? 2u : 1u) * C::kPageBoxBytes);
             const uint32_t dst = sSlots + s * C::kSlotBytes;
-            tma_load_2d(dst, &tm_rope, kDv + 16, pA * kPage, bar(kBarSlotFull + s), pol_rope);
-            if (hasB)
-              tma_load_2d(dst + C::kPageBoxBytes, &tm_rope, kDv + 16, pB * kPage, bar(kBarSlotFull + s), pol_rope);
+            tma_load_2d(dst, &tm_rope, kDv + 16, sp.a * kPage, bar(kBarSlotFull + s), pol_rope);
+            if (sp.has_b)
+              tma_load_2d(dst + C::kPageBoxBytes, &tm_rope, kDv + 16, sp.b * kPage, bar(kBarSlotFull + s), pol_rope);
             last_rope[s] = static_cast<int>(use);
           }
         }
@@ -762,30 +770,25 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
         const int npages = (L + kPage - 1) / kPage;
         const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
         const int n = c1 - c0;
-        uint32_t su_prev = 0;
-        for (int t = 0; t < n && !aborted; ++t) {
-          const int blk = c0 + t;
-          const int t0 = blk * kBlockTokens;
-          const int pA = bt[2 * blk];
-          const bool hasB = 2 * blk + 1 < npages;
-          const int pB = hasB ? bt[2 * blk + 1] : 0;
-          const uint32_t su = us++;
-          ok &= warp_wait(bar(kBarScaleFull + (su & 1u)), (su >> 1) & 1u, wc, lane);
-          for (int grp = 0; grp < 4 && !aborted; ++grp)
-            aborted = !dequant_slot(grp, su & 1u, t0, L);
-          if (aborted) break;
-          rope_slot(pA, pB, hasB);
-          if (t > 0) {
-            for (int grp = 0; grp < 4 && !aborted; ++grp)
-              aborted = !dequant_slot(grp, su_prev & 1u, t0 - kBlockTokens, L);
-            if (!aborted && dt == 0) mbar_arrive(bar(kBarScaleEmpty + (su_prev & 1u)));
+        const uint32_t us0 = us;  // scale fill index of step 0 of this chunk
+        for (int e = 0; !aborted && e < order_len(n); ++e) {
+          bool is_v;
+          int t;
+          order_at(e, n, is_v, t);
+          const int t0 = (c0 + t) * kBlockTokens;
+          const uint32_t su = us0 + static_cast<uint32_t>(t);  // scale fill of step t
+          if (!is_v) {
+            ok &= warp_wait(bar(kBarScaleFull + su % kNumS), (su / kNumS) & 1u, wc, lane);
+            ++us;
           }
-          su_prev = su;
+          for (int grp = 0; grp < 4 && !aborted; ++grp) aborted = !dequant_slot(grp, su % kNumS, t0, L);
+          if (aborted) break;
+          if (!is_v) {
+            rope_slot(step_pages(bt, c0 + t, npages));
+          } else if (dt == 0) {
+            mbar_arrive(bar(kBarScaleEmpty + su % kNumS));  // the last use of step t's scales
+          }
         }
-        if (aborted) break;
-        const int tl = (c1 - 1) * kBlockTokens;
-        for (int grp = 0; grp < 4 && !aborted; ++grp) aborted = !dequant_slot(grp, su_prev & 1u, tl, L);
-        if (!aborted && dt == 0) mbar_arrive(bar(kBarScaleEmpty + (su_prev & 1u)));
       }
       if (dt == 0 && *abort_flag)
         for (int s = 0; s < C::kNumSlots; ++s)
@@ -801,11 +804,11 @@ __global__ void __launch_bounds__(Cfg<RG, RETAIN, FP8>::kThreads, 1)
   }
 }
 
-template <int RG, bool RETAIN, bool FP8>
+template <int RG, bool FP8>
 int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_scale,
                 const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
-  using C = Cfg<RG, RETAIN, FP8>;
-  auto kern = mla_decode_kernel<RG, RETAIN, FP8>;
+  using C = Cfg<RG, FP8>;
+  auto kern = mla_decode_kernel<RG, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid(p.num_sm_parts, p.row_groups, 1);
@@ -818,9 +821,9 @@ int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtenso
 int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, int rows_per_cta,
                        cudaStream_t stream) {
   switch (rows_per_cta) {
-    case 16: return launch_impl<16, false, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
-    case 32: return launch_impl<32, false, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
-    case 64: return launch_impl<64, false, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+    case 16: return launch_impl<16, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+    case 32: return launch_impl<32, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+    case 64: return launch_impl<64, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }
 }
@@ -828,9 +831,9 @@ int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const 
 int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
                       const CUtensorMap& tm_rope, const DecodeParams& p, int rows_per_cta, cudaStream_t stream) {
   switch (rows_per_cta) {
-    case 16: return launch_impl<16, false, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
-    case 32: return launch_impl<32, false, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
-    case 64: return launch_impl<64, false, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
+    case 16: return launch_impl<16, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
+    case 32: return launch_impl<32, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
+    case 64: return launch_impl<64, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }
 }
