@@ -59,6 +59,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32) mla_combine_kernel(const C
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float lse = m + logf(sum);
+  // unrolled so that the loads of several splits are in flight together
+#pragma unroll 4
   for (int s = 0; s < ns; ++s) {
     const float w = expf(p.lse_part[static_cast<long long>(s0 + s) * R + row] - lse);
     const float4* src = reinterpret_cast<const float4*>(p.o_part + (static_cast<long long>(s0 + s) * R + row) * kDv);

@@ -22,6 +22,7 @@ namespace mla {
 namespace {
 
 constexpr int kSchedThreads = 1024;
+constexpr int kSmemBatch = 8192;  // batches up to this size keep the prefix array in shared memory
 
 __device__ __forceinline__ long long blocks_of(int L) { return L > 0 ? (L + kBlockTokens - 1) / kBlockTokens : 0; }
 
@@ -56,8 +57,10 @@ __global__ void __launch_bounds__(kSchedThreads)
     mla_tile_scheduler_kernel(const int32_t* __restrict__ seqlens, int batch, int parts, int32_t* __restrict__ md,
                               int32_t* __restrict__ ns) {
   __shared__ long long warp_tot[32];
+  __shared__ int32_t s_cum[kSmemBatch + 1];  // C_{b+1}: binary searches stay on chip
   const long long F = kFixedSplitCost;
   const int tid = threadIdx.x;
+  const bool on_chip = batch <= kSmemBatch;
 
   // pass 1: ns[b + 1] = C_{b+1} (inclusive prefix of costs), T
   long long carry = 0;
@@ -66,20 +69,27 @@ __global__ void __launch_bounds__(kSchedThreads)
     const long long n = b < batch ? blocks_of(seqlens[b]) : 0;
     long long tile_total;
     const long long incl = block_scan(n > 0 ? n + F : 0, warp_tot, &tile_total) + carry;
-    if (b < batch) ns[b + 1] = static_cast<int32_t>(incl);
+    if (b < batch) {
+      ns[b + 1] = static_cast<int32_t>(incl);
+      if (on_chip) s_cum[b + 1] = static_cast<int32_t>(incl);
+    }
     carry += tile_total;
   }
-  if (tid == 0) ns[0] = 0;
+  if (tid == 0) {
+    ns[0] = 0;
+    s_cum[0] = 0;
+  }
   const long long T = carry;
   const long long q = T > 0 ? (T + parts - 1) / parts : 1;
   __syncthreads();
 
   // pass 2: per part, the first block at a position >= x (binary search on C_{b+1})
+  const int32_t* cum = on_chip ? s_cum : ns;  // C_{b+1} at index b + 1
   auto find = [&](long long x, int& fb, int& fj) {
     int lo = 0, hi = batch;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (static_cast<long long>(ns[mid + 1]) > x) hi = mid;
+      if (static_cast<long long>(cum[mid + 1]) > x) hi = mid;
       else lo = mid + 1;
     }
     fb = lo;
@@ -87,7 +97,7 @@ __global__ void __launch_bounds__(kSchedThreads)
       fj = 0;
       return;
     }
-    const long long cb = lo == 0 ? 0 : ns[lo];
+    const long long cb = lo == 0 ? 0 : cum[lo];
     const long long j = x - (cb + F);
     fj = j > 0 ? static_cast<int>(j) : 0;
   };
@@ -97,7 +107,7 @@ __global__ void __launch_bounds__(kSchedThreads)
     find(static_cast<long long>(p + 1) * q, eb, ej);
     int ordinal = 0;
     if ((bb != eb || bj != ej) && bb < batch) {
-      const long long cb = bb == 0 ? 0 : ns[bb];
+      const long long cb = bb == 0 ? 0 : cum[bb];
       ordinal = static_cast<int>(p - (cb + F) / q);
     }
     int32_t* row = md + static_cast<long long>(p) * kMdInts;

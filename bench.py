@@ -139,6 +139,12 @@ def oracle_baseline(case, budget_s: float = 15.0):
     return {"seconds": dt, "requests": len(done), "units": units, "cores": int(cores)}
 
 
+# DRAM bytes (read + write) per launch of the main kernel from an ncu capture of the current
+# kernel, scaled to the full workload by the KV bytes it processes (see profiles/); None when
+# the kernel has changed since the counters were taken.
+TRAFFIC = {"mem_b128_h16_L8192": 1250.5e6}
+
+
 def rank_case(workload: str, rank: int, batch=None):
     """The batch of requests rank `rank` owns: the named workload's shapes and cache lengths,
     with the random contents drawn from a seed shifted by the rank (independent problems)."""
@@ -316,7 +322,11 @@ def main():
     total_bytes = units["bytes"] * world * args.steps
     value = total_bytes / (ms_total * 1e-3) / 1e9
     tflops = units["flops"] * world * args.steps / (ms_total * 1e-3) / 1e12
-    achieved = units["bytes"] / (decode_ms * 1e-3) / 1e9
+    hbm_bound = units["bytes"] / (hbm_peak * 1e9) >= units["flops"] / (tc_peak * 1e12)
+    if hbm_bound:
+        achieved, peak, runit = units["bytes"] / (decode_ms * 1e-3) / 1e9, hbm_peak, "GB/s"
+    else:
+        achieved, peak, runit = units["flops"] / (decode_ms * 1e-3) / 1e12, tc_peak, "TFLOP/s"
     roof_time = max(units["bytes"] / (hbm_peak * 1e9), units["flops"] / (tc_peak * 1e12))
     line = {
         "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -328,11 +338,10 @@ def main():
                    "parallelism": f"replicas x{world} (independent requests per GPU)"},
         "tflops": tflops,
         "roofline_fraction": roof_time / (ms_total / args.steps * 1e-3),
-        "roofline": {"bound": "hbm" if units["bytes"] / (hbm_peak * 1e9) >= units["flops"] / (tc_peak * 1e12)
-                     else "tensor",
+        "roofline": {"bound": "hbm" if hbm_bound else "tensor",
                      "kernel": "mla_decode_kvcache (split-KV main + combine)", "achieved": achieved,
-                     "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": None,
-                     "peak_kind": peak_kind},
+                     "peak": peak, "unit": runit, "frac": achieved / peak, "traffic": TRAFFIC.get(args.workload),
+                     "peak_kind": peak_kind + (" copy bandwidth" if hbm_bound else " cuBLAS bf16 burst")},
         "e2e": None if e2e_ms is None else {
             "value": units["bytes"] * world * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
