@@ -81,7 +81,7 @@ int mla_num_sm_parts(int rows_per_kv_head, int h_kv, int device) {
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms < 1)
     return MLA_ERR_NO_DEVICE;
-  const int g = mla::row_groups_for(rows_per_kv_head);
+  const int g = mla::sms_per_part(rows_per_kv_head);
   const int parts = sms / (h_kv * g);
   return parts < 1 ? 1 : parts;
 }
@@ -126,7 +126,8 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
 
   EncodeTiledFn encode = encode_fn();
   if (!encode) return MLA_ERR_CUDA;
-  const int rg = rows_per_cta_for(rows);
+  const bool pair = mla::use_pair_kernel(rows, kv_dtype == MLA_KV_FP8);
+  const int rg = pair ? mla::kRowsPerCta : rows_per_cta_for(rows);  // query rows of one Q box
 
   // q as a 3-D tensor {576 dims, rows, batch}; one box = 64 dims x rg rows of one request
   CUtensorMap tm_q, tm_kv, tm_scale, tm_rope;
@@ -188,13 +189,14 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   p.s_q = s_q;
   p.h_q = h_q;
   p.rows = rows;
-  p.row_groups = (rows + rg - 1) / rg;
+  p.row_groups = pair ? (rows + mla::kPairRows - 1) / mla::kPairRows : (rows + rg - 1) / rg;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = kv_dtype == MLA_KV_BF16 ? mla::launch_decode_bf16(tm_q, tm_kv, p, rg, st)
-                                  : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, rg, st);
+  int e = pair                      ? mla::launch_decode_pair_bf16(tm_q, tm_kv, p, st)
+          : kv_dtype == MLA_KV_BF16 ? mla::launch_decode_bf16(tm_q, tm_kv, p, rg, st)
+                                    : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
 
   mla::CombineParams cp{};

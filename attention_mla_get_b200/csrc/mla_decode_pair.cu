@@ -1,0 +1,741 @@
+// Split-KV MLA decode on CTA pairs (cta_group::2) for requests with more than 64 query rows,
+// bf16 paged KV cache.
+//
+// The problem is the one of mla_decode.cu (FlashMLA pages: mha_fwd_kvcache_mla on a paged
+// latent cache of 576-dim tokens, V = the first 512 dims, 64-token pages addressed by
+// block_table).  With many query rows per request (h_q = 128 query heads sharing one latent KV
+// head, "MLA" on the deepseekonline.chat page) the work per cached token is large, so the
+// kernel is bound by the tensor core, and what limits it is how many bytes the SMs must read
+// per MMA.  A 2-SM pair handles 128 query rows and 256 tokens per step:
+//
+//   S^T [256 tokens x 128 rows]  = K[256 x 576] . Q^T[576 x 128]        M = 256, N = 128
+//   O^T [512 dims  x 128 rows]  += V^T[512 x 256] . P^T[256 x 128]      2 x (M = 256, N = 128)
+//
+// Each MMA of the pair runs at the full per-SM rate (N = 128), each CTA keeps only its 64 rows
+// of Q^T (N half) and of P^T, and each SM's tensor memory holds the pair's M half: S^T of its own
+// 128 tokens and O^T of its own 256 output dims (dims 128c..128c+127 and 256+128c..256+128c+127
+// on CTA c).  That is 2 x 128 + 2 x 128 of the 512 TMEM columns, so the whole 512 x 128 output
+// of a 128-row group stays on chip.
+//
+// Data per step and CTA c: the 9 K boxes (64 dims x 128 tokens) of its own 128-token block for
+// S^T, and the V boxes (its 256 dims x all 256 tokens) for O^T, read through the block table
+// with 64-token TMA boxes (the 9-boxes-per-page split of the wmrh.cn page, "内存访问优化策略").
+// Both CTAs' loads count their bytes on the leader's (rank 0) barrier; the leader's MMA
+// thread issues the pair MMAs; tcgen05.commit multicasts completion to both CTAs.
+//
+// Online softmax (the running-max-and-rescale idea of the wmrh.cn page, "跷跷板调度算法"):
+// CTA c sees only its own 128 tokens of S^T, so the per-row block maximum is exchanged through
+// distributed shared memory every step, and both CTAs make the same rescale decisions.  Each
+// CTA writes the bf16 P^T rows of its tokens into both CTAs' P^T halves (64 query rows each).
+// Row sums are exchanged once per chunk.
+//
+// Ring: 16 KB slots (K slot = 128 tokens x 64 dims, V slot = one page x 128 dims).  Order per
+// chunk of n pair steps: K(0), K(1), then V(t), K(t + 2) for t = 0 .. n-1 (QK runs one step
+// ahead of PV).  Tokens past the request or the chunk are masked in S^T; their V rows (stale
+// ring contents or the cache's unused page tail) are zeroed by the leader before PV reads them.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "mla_internal.h"
+#include "mla_ptx.cuh"
+
+namespace mla {
+
+namespace {
+
+constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr int kThreads = 320;     // warps 0-7 softmax + epilogue, 8 producer, 9 MMA / TMEM owner
+constexpr int kSoftmaxThreads = 256;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr int kRows = 128;        // query rows per pair
+constexpr int kHalfRows = 64;     // query rows of Q^T / P^T held by each CTA
+constexpr int kNumSlots = 7;
+constexpr int kSlotBytes = 16384;
+constexpr int kBoxBytes = 8192;   // 64 tokens x 64 dims bf16
+constexpr int kKFills = 9;        // K slots per step (576 dims / 64)
+constexpr int kVFills = 8;        // V slots per step (2 dim blocks x 4 pages)
+constexpr int kQBytes = 9 * kBoxBytes;          // 64 rows x 576 dims
+constexpr int kPBytes = 256 * kHalfRows * 2;    // 256 tokens x 64 rows bf16
+constexpr int kOffQ = 0;
+constexpr int kOffP = kOffQ + kQBytes;
+constexpr int kOffSlots = kOffP + kPBytes;
+constexpr int kOffMisc = kOffSlots + kNumSlots * kSlotBytes;
+constexpr int kMiscBytes = 6144;
+constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+constexpr int kTmemCols = 512;
+constexpr int kColO = 0;      // O^T dim block m at columns 128m
+constexpr int kColS = 256;    // S^T buffer sb at columns 256 + 128 sb
+constexpr uint32_t kIdescQK = idesc_bf16(256, kRows, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16(256, kRows, true, true);
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffP % 1024 == 0 && kOffSlots % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+
+// misc area: barriers, then scalars, then per-row scratch
+enum : int {
+  kBarSlotFull = 0,                      // [kNumSlots] leader: both producers, count 2 + bytes
+  kBarSlotEmpty = kBarSlotFull + kNumSlots,   // [kNumSlots] both: pair commit
+  kBarZFull = kBarSlotEmpty + kNumSlots,      // [kNumSlots] leader: V rows of a tail step zeroed
+  kBarSFull = kBarZFull + kNumSlots,          // [2] both: pair commit
+  kBarSEmpty = kBarSFull + 2,                 // [2] leader: 16 softmax warps of the pair
+  kBarPFull = kBarSEmpty + 2,                 // leader: the 8 warps that write P^T locally
+  kBarPEmpty = kBarPFull + 1,                 // both: pair commit
+  kBarQFull = kBarPEmpty + 1,                 // leader: both producers
+  kBarQEmpty = kBarQFull + 1,                 // both: pair commit
+  kBarOFull = kBarQEmpty + 1,                 // both: pair commit
+  kBarOEmpty = kBarOFull + 1,                 // leader: 16 epilogue warps
+  kBarDrain = kBarOEmpty + 1,                 // leader: final commit
+  kBarMaxFull = kBarDrain + 1,                // [2] both: 512 bytes of the peer's block maxima
+  kBarLFull = kBarMaxFull + 2,                // both: 512 bytes of the peer's row sums
+  kBarPRecv = kBarLFull + 1,                  // both: 16 KB of P^T rows from the peer
+  kNumBars = kBarPRecv + 1,
+};
+constexpr int kMiscHolder = 512;   // TMEM base address
+constexpr int kMiscAbort = 516;    // abort flag
+constexpr int kMiscPeerFills = 520;// follower's slot fills (written into the leader at exit)
+constexpr int kMiscPeerQ = 524;    // follower's Q fills
+constexpr int kMiscRed = 1024;     // float [4 lane quadrants][128 rows]
+constexpr int kMiscM = 3072;       // float [128]
+constexpr int kMiscAlpha = 3584;   // float [128]
+constexpr int kMiscInv = 4096;     // float [128]
+constexpr int kMiscXMax = 4608;    // float [2][128]: the peer's block maxima
+constexpr int kMiscXL = 5632;      // float [128]: the peer's row sums
+static_assert(kNumBars * 8 <= kMiscHolder, "barrier area");
+static_assert(kMiscXL + 512 <= kMiscBytes, "misc area");
+
+__device__ __forceinline__ int blocks_of(int L) { return L > 0 ? (L + kBlockTokens - 1) / kBlockTokens : 0; }
+
+struct ChunkWalk {
+  int b, blk, split, end_b, end_blk;
+  __device__ ChunkWalk(const DecodeParams& p, int part) {
+    const int32_t* md = p.tile_md + part * kMdInts;
+    b = md[0];
+    blk = md[1];
+    end_b = md[2];
+    end_blk = md[3];
+    split = md[4];
+  }
+  __device__ bool next(const DecodeParams& p, int& cb, int& c0, int& c1, int& csplit) {
+    while (b < end_b || (b == end_b && blk < end_blk)) {
+      const int n = blocks_of(p.cache_seqlens[b]);
+      const int stop = (b == end_b) ? end_blk : n;
+      cb = b;
+      c0 = blk;
+      c1 = stop;
+      csplit = split;
+      ++b;
+      blk = 0;
+      if (b <= p.batch) split = p.num_splits[b];
+      if (stop > c0) return true;
+    }
+    return false;
+  }
+};
+
+// Fill / consume order of a chunk of n pair steps: K(0), K(1), then V(t), K(t + 2).
+__device__ __forceinline__ void order_at(int e, int n, bool& is_v, int& step) {
+  const int head = min(2, n);
+  if (e < head) {
+    is_v = false;
+    step = e;
+    return;
+  }
+  const int r = e - head;
+  const int tail_k = n - head;
+  if (r < 2 * tail_k) {
+    is_v = (r & 1) == 0;
+    step = is_v ? (r >> 1) : (r >> 1) + head;
+  } else {
+    is_v = true;
+    step = tail_k + (r - 2 * tail_k);
+  }
+}
+// Slot fills of the chunk before the first V slot of step t.
+__device__ __forceinline__ uint32_t fills_before_v(int t, int n) {
+  return static_cast<uint32_t>(kKFills * min(t + 2, n) + kVFills * t);
+}
+// Step t of a chunk [c0, c1) reads tokens no request position covers (V rows must be zeroed).
+__device__ __forceinline__ bool is_tail(int c0, int c1, int t, int L) {
+  return (c0 + 2 * t + 1 >= c1) || ((c0 + 2 * t + 2) * kBlockTokens > L);
+}
+
+// Bounded waits (cluster-scope acquire).  On time-out: status bit, this CTA's and the peer's
+// abort flags; every waiter of both CTAs then unwinds.
+struct PairCtl {
+  volatile int* abort_flag;
+  uint32_t peer_abort;  // cluster address of the peer's abort flag
+  int* status;
+};
+
+static __device__ __noinline__ void pair_timeout(const PairCtl& c) {
+  *c.abort_flag = 1;
+  st_cluster_u32(c.peer_abort, 1u);
+  if (c.status) atomicOr(c.status, kStatusWaitTimeout);
+  __threadfence();
+}
+
+__device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, const PairCtl& c) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*c.abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      pair_timeout(c);
+      return false;
+    }
+  }
+}
+
+// used only at exit: bounded, ignores the abort flag
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) return;
+  }
+}
+
+__device__ __forceinline__ bool warp_pwait(uint32_t bar, uint32_t parity, const PairCtl& c, int lane) {
+  int ok = 1;
+  if (lane == 0) ok = pwait(bar, parity, c) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Warp reduce-scatter (sum) of 64 column values over the 32 token lanes: afterwards lane l
+// holds the warp-wide sums of columns 2l and 2l + 1 in v[0], v[1].
+__device__ __forceinline__ void reduce_scatter64_sum(float* v, int lane) {
+#pragma unroll
+  for (int r = 0; r < 5; ++r) {
+    const int o = 16 >> r;
+    const int n = 64 >> r;
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float keep = upper ? v[i + n / 2] : v[i];
+      const float send = upper ? v[i] : v[i + n / 2];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                           const DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + kOffQ;
+  const uint32_t sP = sbase + kOffP;
+  const uint32_t sSlots = sbase + kOffSlots;
+  uint8_t* misc = smem + kOffMisc;
+  const uint32_t sMisc = smem_u32(misc);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + kMiscHolder);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + kMiscAbort);
+  float* red = reinterpret_cast<float*>(misc + kMiscRed);
+  float* m_sm = reinterpret_cast<float*>(misc + kMiscM);
+  float* alpha_sm = reinterpret_cast<float*>(misc + kMiscAlpha);
+  float* inv_sm = reinterpret_cast<float*>(misc + kMiscInv);
+  const float* xmax = reinterpret_cast<const float*>(misc + kMiscXMax);
+  const float* xl = reinterpret_cast<const float*>(misc + kMiscXL);
+  auto bar = [&](int i) -> uint32_t { return sMisc + 8u * static_cast<uint32_t>(i); };
+
+  const uint32_t rank = cluster_cta_rank();
+  const uint32_t peer = rank ^ 1u;
+  const bool leader = rank == 0;
+  auto lead = [&](uint32_t a) -> uint32_t { return map_to_cta(a, 0); };
+  auto other = [&](uint32_t a) -> uint32_t { return map_to_cta(a, peer); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int part = blockIdx.x >> 1;
+  const int rg = blockIdx.y;  // 128-row group
+  const PairCtl wc{abort_flag, other(sMisc + kMiscAbort), p.status};
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNumSlots; ++i) {
+      mbar_init(bar(kBarSlotFull + i), 2);
+      mbar_init(bar(kBarSlotEmpty + i), 1);
+      mbar_init(bar(kBarZFull + i), 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarSEmpty + i), 16);
+      mbar_init(bar(kBarMaxFull + i), 1);
+    }
+    mbar_init(bar(kBarPFull), 8);
+    mbar_init(bar(kBarPRecv), 1);
+    mbar_init(bar(kBarPEmpty), 1);
+    mbar_init(bar(kBarQFull), 2);
+    mbar_init(bar(kBarQEmpty), 1);
+    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarOEmpty), 16);
+    mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarLFull), 1);
+    *abort_flag = 0;
+    *reinterpret_cast<uint32_t*>(misc + kMiscPeerFills) = 0;
+    *reinterpret_cast<uint32_t*>(misc + kMiscPeerQ) = 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kv);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  pdl_launch_dependents();
+
+  // state the exit sequence needs
+  uint32_t fills = 0;  // producer: slot fills issued
+  int q_fills = 0;     // producer: Q fills issued
+
+  if (warp == kWarpProducer) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+      const uint64_t pol_v = p.row_groups > 1 ? pol_keep : pol_stream;
+      const uint64_t pol_rope = p.row_groups > 1 ? pol_keep : pol_stream;
+      int last_use[kNumSlots];
+      for (int i = 0; i < kNumSlots; ++i) last_use[i] = -1;
+      bool ok = true;
+      ChunkWalk walk(p, part);
+      int b, c0, c1, split;
+      // two 64x64 boxes into one slot: (x0, y0) at +0 and (x1, y1) at +8 KB, each only if valid
+      auto fill = [&](int x0, int y0, bool v0, int x1, int y1, bool v1, uint64_t pol) -> bool {
+        const int s = static_cast<int>(fills % kNumSlots);
+        const uint32_t use = fills / kNumSlots;
+        if (!pwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
+        const uint32_t full = lead(bar(kBarSlotFull + s));
+        mbar_arrive_expect_tx_relaxed(full, static_cast<uint32_t>(((v0 ? 1 : 0) + (v1 ? 1 : 0)) * kBoxBytes));
+        const uint32_t dst = sSlots + static_cast<uint32_t>(s) * kSlotBytes;
+        if (v0) tma_load_2d_pair(dst, &tm_kv, x0, y0, full, pol);
+        if (v1) tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x1, y1, full, pol);
+        last_use[s] = static_cast<int>(use);
+        ++fills;
+        return true;
+      };
+      while (ok && walk.next(p, b, c0, c1, split)) {
+        const int L = p.cache_seqlens[b];
+        const int npages = (L + kPage - 1) / kPage;
+        const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
+        if (!pwait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc)) break;
+        const uint32_t qfull = lead(bar(kBarQFull));
+        mbar_arrive_expect_tx_relaxed(qfull, static_cast<uint32_t>(kQBytes));
+        for (int a = 0; a < 9; ++a)
+          tma_load_3d_pair(sQ + a * kBoxBytes, &tm_q, 64 * a, rg * kRows + static_cast<int>(rank) * kHalfRows, b,
+                           qfull);
+        ++q_fills;
+        const int n = (c1 - c0 + 1) / 2;
+        for (int e = 0; ok && e < 2 * n; ++e) {
+          bool is_v;
+          int t;
+          order_at(e, n, is_v, t);
+          if (!is_v) {
+            // K(t): this CTA's own 128-token block, all 576 dims
+            const int kb = c0 + 2 * t + static_cast<int>(rank);
+            const bool va = kb < c1;
+            const bool vb = va && (2 * kb + 1 < npages);
+            const int ya = va ? bt[2 * kb] * kPage : 0;
+            const int yb = vb ? bt[2 * kb + 1] * kPage : 0;
+            for (int j = 0; ok && j < kKFills; ++j)
+              ok = fill(64 * j, ya, va, 64 * j, yb, vb, j < 8 ? pol_keep : pol_rope);
+          } else {
+            // V(t): this CTA's 256 output dims of all four pages of the step
+            for (int m = 0; ok && m < 2; ++m) {
+              const int d = 256 * m + 128 * static_cast<int>(rank);
+              for (int q = 0; ok && q < 4; ++q) {
+                const int pg = 2 * (c0 + 2 * t) + q;
+                const bool v = (c0 + 2 * t + (q >> 1) < c1) && pg < npages;
+                const int y = v ? bt[pg] * kPage : 0;
+                ok = fill(d, y, v, d + 64, y, v, pol_v);
+              }
+            }
+          }
+        }
+      }
+      if (!*abort_flag) {
+        // the last pair commits on this CTA's barriers have landed before it may exit
+        for (int s = 0; s < kNumSlots; ++s)
+          if (last_use[s] >= 0) drain_wait(bar(kBarSlotEmpty + s), static_cast<uint32_t>(last_use[s]) & 1u);
+        if (q_fills > 0) drain_wait(bar(kBarQEmpty), static_cast<uint32_t>(q_fills - 1) & 1u);
+      }
+      if (!leader) {
+        st_cluster_u32(lead(sMisc + kMiscPeerFills), fills);
+        st_cluster_u32(lead(sMisc + kMiscPeerQ), static_cast<uint32_t>(q_fills));
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ================================ MMA issuer (leader) =========================
+    if (leader && lane == 0) {
+      uint32_t g = 0;   // slot fills consumed
+      uint32_t u = 0;   // QK steps issued
+      uint32_t up = 0;  // PV steps issued
+      uint32_t zpar = 0;
+      int chunk = 0;
+      bool ok = true;
+      ChunkWalk walk(p, part);
+      int b, c0, c1, split;
+      auto next_slot = [&](uint32_t& s) -> bool {
+        s = g % kNumSlots;
+        if (!pwait(bar(kBarSlotFull + s), (g / kNumSlots) & 1u, wc)) return false;
+        ++g;
+        tc_fence_after();
+        return true;
+      };
+      while (ok && walk.next(p, b, c0, c1, split)) {
+        const int L = p.cache_seqlens[b];
+        const int n = (c1 - c0 + 1) / 2;
+        if (!pwait(bar(kBarQFull), chunk & 1, wc)) break;
+        for (int e = 0; ok && e < 2 * n; ++e) {
+          bool is_v;
+          int t;
+          order_at(e, n, is_v, t);
+          if (!is_v) {
+            const int sb = static_cast<int>(u & 1u);
+            if (!pwait(bar(kBarSEmpty + sb), ((u >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d = tmem + kColS + 128u * sb;
+            for (int j = 0; ok && j < kKFills; ++j) {
+              uint32_t s;
+              if (!next_slot(s)) { ok = false; break; }
+              const uint32_t kbase = sSlots + s * kSlotBytes;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16_pair(d, smem_desc(kbase + 32 * kk, 16, 1024, kSwizzle128),
+                               smem_desc(sQ + j * kBoxBytes + 32 * kk, 16, 1024, kSwizzle128), kIdescQK,
+                               (j | kk) != 0 ? 1u : 0u);
+              umma_commit_pair_mc(bar(kBarSlotEmpty + s), 0x3);
+            }
+            if (!ok) break;
+            umma_commit_pair_mc(bar(kBarSFull + sb), 0x3);
+            ++u;
+            if (t == n - 1) umma_commit_pair_mc(bar(kBarQEmpty), 0x3);
+          } else {
+            if (!pwait(bar(kBarPFull), up & 1u, wc)) { ok = false; break; }
+            if (t == 0 && !pwait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            const bool tail = is_tail(c0, c1, t, L);
+            for (int m = 0; ok && m < 2; ++m) {
+              for (int q = 0; q < 4; ++q) {
+                uint32_t s;
+                if (!next_slot(s)) { ok = false; break; }
+                if (tail) {
+                  if (!pwait(bar(kBarZFull + s), (zpar >> s) & 1u, wc)) { ok = false; break; }
+                  zpar ^= 1u << s;
+                  tc_fence_after();
+                }
+                const uint32_t vbase = sSlots + s * kSlotBytes;
+#pragma unroll
+                for (int kt = 0; kt < 4; ++kt)
+                  umma_bf16_pair(tmem + kColO + 128u * m, smem_desc(vbase + 2048 * kt, kBoxBytes, 1024, kSwizzle128),
+                                 smem_desc(sP + (64 * q + 16 * kt) * 128, kBoxBytes, 1024, kSwizzle128), kIdescPV,
+                                 (t == 0 && q == 0 && kt == 0) ? 0u : 1u);
+                umma_commit_pair_mc(bar(kBarSlotEmpty + s), 0x3);
+              }
+            }
+            if (!ok) break;
+            umma_commit_pair_mc(bar(kBarPEmpty), 0x3);
+            ++up;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(bar(kBarOFull), 0x3);
+        ++chunk;
+      }
+      // every pair MMA is complete before tensor memory is released
+      umma_commit_pair(bar(kBarDrain));
+      drain_wait(bar(kBarDrain), 0);
+    }
+  } else {
+    // ============================ softmax + epilogue ==============================
+    // Warp w reads TMEM lane quadrant qd = w % 4 (tokens 32qd..32qd+31 of this CTA's block, or
+    // output dims of O^T) and column half h = w / 4 (query rows 64h..64h+63 of S^T; O^T block m = h).
+    // Threads 0..127 also own one query row each for the running max and the row sums.
+    const int tid = threadIdx.x;  // 0..255
+    const int qd = warp & 3;
+    const int h = warp >> 2;
+    const int tl = 32 * qd + lane;  // token lane of S^T, dim lane of O^T
+    const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+    const float NEG_INF = -CUDART_INF_F;
+    float m_ref = NEG_INF;  // row tid (tid < 128): reference max, log2 units
+    float lsum[2] = {0.f, 0.f};
+    uint32_t u = 0;
+    uint32_t gchunk = 0;
+    int chunk = 0;
+    bool fail = false;
+    const int R = p.rows;
+    const int row0 = rg * kRows;
+    ChunkWalk walk(p, part);
+    int b, c0, c1, split;
+    while (walk.next(p, b, c0, c1, split)) {
+      const int L = p.cache_seqlens[b];
+      const int n = (c1 - c0 + 1) / 2;
+      const bool single = (p.num_splits[b + 1] - p.num_splits[b]) == 1;
+      bool aborted = false;
+      for (int t = 0; t < n; ++t) {
+        const int kb = c0 + 2 * t + static_cast<int>(rank);
+        const int j = kb * kBlockTokens + tl;
+        const int sb = static_cast<int>(u & 1u);
+        bool ok = warp_pwait(bar(kBarSFull + sb), (u >> 1) & 1u, wc, lane);
+        float x[64];
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) tmem_ld16(tmem + lane_base + kColS + 128u * sb + 64u * h + c, x + c);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(lead(bar(kBarSEmpty + sb)));
+        // key j is visible to row r iff j < L, its block is in this chunk and, when causal,
+        // j <= L - s_q + r / h_q, i.e. r >= (j - L + s_q) * h_q
+        int cmin = -(1 << 30);
+        if (p.causal) {
+          const int i0 = j - L + p.s_q;
+          if (i0 > 0) cmin = i0 * p.h_q - row0 - 64 * h;
+        }
+        if (kb >= c1 || j >= L) cmin = 1 << 30;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[c] = (c >= cmin) ? x[c] * p.scale_log2 : NEG_INF;
+        // column maxima over this warp's 32 tokens; lane l keeps columns l and 32 + l
+        float k0 = NEG_INF, k1 = NEG_INF;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float m0 = warp_max_f32(x[c]);
+          const float m1 = warp_max_f32(x[32 + c]);
+          k0 = (lane == c) ? m0 : k0;
+          k1 = (lane == c) ? m1 : k1;
+        }
+        red[qd * kRows + 64 * h + lane] = k0;
+        red[qd * kRows + 64 * h + 32 + lane] = k1;
+        if (named_bar_any(1, kSoftmaxThreads, !ok || fail)) { aborted = true; break; }
+        bool need = false;
+        if (tid < kRows) {
+          // block max of row tid over this CTA's tokens, then over the pair's
+          const float bm_own =
+              fmaxf(fmaxf(red[tid], red[kRows + tid]), fmaxf(red[2 * kRows + tid], red[3 * kRows + tid]));
+          const uint32_t xb = u & 1u;
+          st_async_f32(other(sMisc + kMiscXMax + 4u * (xb * kRows + tid)), bm_own, other(bar(kBarMaxFull + xb)));
+          if (tid == 0) mbar_arrive_expect_tx(bar(kBarMaxFull + xb), 4u * kRows);
+          ok &= pwait(bar(kBarMaxFull + xb), (u >> 1) & 1u, wc);
+          const float bm = fmaxf(bm_own, xmax[xb * kRows + tid]);
+          float alpha = 1.f;
+          float m_new = m_ref;
+          if (bm > m_ref + kTau || (m_ref == NEG_INF && bm != NEG_INF)) {
+            m_new = bm;
+            alpha = (m_ref == NEG_INF) ? 0.f : ex2(m_ref - m_new);
+          }
+          need = (alpha != 1.f) && (t > 0);
+          m_ref = m_new;
+          m_sm[tid] = (m_new == NEG_INF) ? 0.f : m_new;
+          alpha_sm[tid] = alpha;
+        }
+        const bool rescale = named_bar_any(1, kSoftmaxThreads, need);
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(m_sm + 64 * h + c);
+          x[c + 0] = ex2(x[c + 0] - m4.x);
+          x[c + 1] = ex2(x[c + 1] - m4.y);
+          x[c + 2] = ex2(x[c + 2] - m4.z);
+          x[c + 3] = ex2(x[c + 3] - m4.w);
+        }
+        {
+          float v[64];
+#pragma unroll
+          for (int c = 0; c < 64; ++c) v[c] = x[c];
+          reduce_scatter64_sum(v, lane);  // lane l: columns 2l, 2l + 1
+#pragma unroll
+          for (int i = 0; i < 2; ++i) lsum[i] = lsum[i] * alpha_sm[64 * h + 2 * lane + i] + v[i];
+        }
+        // P^T of step u - 1 has been read (and O^T is final for it) once PEmpty flips
+        if (u >= 1) ok &= warp_pwait(bar(kBarPEmpty), (u - 1) & 1u, wc, lane);
+        if (rescale) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < kRows; c += 16) {
+            float o[16];
+            const uint32_t ta = tmem + lane_base + kColO + 128u * h + c;
+            tmem_ld16(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] *= alpha_sm[c + e];
+            tmem_st16(ta, o);
+          }
+          tmem_wait_st();
+        }
+        // this token's P^T row for query rows 64h..64h+63 goes to CTA h's half of P^T
+        const uint32_t T = rank * 128u + static_cast<uint32_t>(tl);
+        const bool local = static_cast<uint32_t>(h) == rank;
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+          const uint32_t off = T * 128u + ((static_cast<uint32_t>(q8) ^ (T & 7u)) << 4);
+          const float* xs = x + 8 * q8;
+          const uint32_t w0 = pack_bf16x2(xs[0], xs[1]), w1 = pack_bf16x2(xs[2], xs[3]);
+          const uint32_t w2 = pack_bf16x2(xs[4], xs[5]), w3 = pack_bf16x2(xs[6], xs[7]);
+          if (local) st_shared_v4(sP + off, w0, w1, w2, w3);
+          else st_async_v4(other(sP + off), w0, w1, w2, w3, other(bar(kBarPRecv)));
+        }
+        if (local) {
+          // this CTA's half of P^T: own rows written here, the peer's rows by st.async (PRecv)
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          int okp = 1;
+          if (lane == 0) {
+            if (qd == 0) mbar_arrive_expect_tx(bar(kBarPRecv), 16384u);
+            okp = pwait(bar(kBarPRecv), u & 1u, wc) ? 1 : 0;
+            fence_proxy_async_smem();
+            mbar_arrive_remote(lead(bar(kBarPFull)));
+          }
+          ok &= __shfl_sync(0xffffffffu, okp, 0) != 0;
+        }
+        if (leader && tid < kRows && is_tail(c0, c1, t, L)) {
+          // zero, in both CTAs' V slots of this step, the rows of tokens outside the request or
+          // the chunk (the leader's full barrier counts both CTAs' bytes)
+          const int r = tid & 63, box = tid >> 6;
+          for (int k = 0; k < kVFills; ++k) {
+            const uint32_t gv = gchunk + fills_before_v(t, n) + static_cast<uint32_t>(k);
+            const uint32_t s = gv % kNumSlots;
+            ok &= warp_pwait(bar(kBarSlotFull + s), (gv / kNumSlots) & 1u, wc, lane);
+            const int q = k & 3;
+            const int jj = (c0 + 2 * t) * kBlockTokens + 64 * q + r;
+            if ((c0 + 2 * t + (q >> 1) >= c1) || jj >= L) {
+              const uint32_t row = sSlots + s * kSlotBytes + static_cast<uint32_t>(box * kBoxBytes + r * 128);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                st_shared_v4(row + 16u * c, 0u, 0u, 0u, 0u);
+                st_cluster_v4(other(row + 16u * c), 0u, 0u, 0u, 0u);
+              }
+            }
+            fence_proxy_async_cluster();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lead(bar(kBarZFull + s)));
+          }
+        }
+        fail |= !ok;
+        ++u;
+      }
+      if (aborted) break;
+      // ------------------------------- epilogue ---------------------------------
+#pragma unroll
+      for (int i = 0; i < 2; ++i) red[qd * kRows + 64 * h + 2 * lane + i] = lsum[i];
+      if (named_bar_any(1, kSoftmaxThreads, fail)) break;
+      bool ok = true;
+      if (tid < kRows) {
+        const float l_own = red[tid] + red[kRows + tid] + red[2 * kRows + tid] + red[3 * kRows + tid];
+        st_async_f32(other(sMisc + kMiscXL + 4u * tid), l_own, other(bar(kBarLFull)));
+        if (tid == 0) mbar_arrive_expect_tx(bar(kBarLFull), 4u * kRows);
+        ok = pwait(bar(kBarLFull), chunk & 1, wc);
+        const float l = l_own + xl[tid];
+        const int row = row0 + tid;
+        const float lse_val = l > 0.f ? (m_ref + log2f(l)) * kLn2 : NEG_INF;
+        inv_sm[tid] = l > 0.f ? 1.f / l : 0.f;
+        if (leader && row < R) {
+          if (single)
+            p.lse[(static_cast<long long>(b) * p.h_q + row % p.h_q) * p.s_q + row / p.h_q] = lse_val;
+          else
+            p.lse_part[static_cast<long long>(split) * R + row] = lse_val;
+        }
+        m_ref = NEG_INF;
+      }
+      lsum[0] = lsum[1] = 0.f;
+      named_bar_sync(1, kSoftmaxThreads);
+      ok &= warp_pwait(bar(kBarOFull), chunk & 1, wc, lane);
+      fail |= !ok;
+      tc_fence_after();
+      {
+        const int dim = 256 * h + 128 * static_cast<int>(rank) + tl;
+#pragma unroll
+        for (int c = 0; c < kRows; c += 16) {
+          float o[16];
+          tmem_ld16(tmem + lane_base + kColO + 128u * h + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int row = row0 + c + e;
+            if (row < R) {
+              const float val = o[e] * inv_sm[c + e];
+              if (single)
+                p.out[(static_cast<long long>(b) * R + row) * kDv + dim] = __float2bfloat16_rn(val);
+              else
+                p.o_part[(static_cast<long long>(split) * R + row) * kDv + dim] = val;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead(bar(kBarOEmpty)));
+      gchunk += static_cast<uint32_t>(kKFills + kVFills) * static_cast<uint32_t>(n);
+      ++chunk;
+    }
+    // the last PEmpty commit on this CTA's barrier has landed before it may exit
+    if (!*abort_flag && u >= 1 && lane == 0) drain_wait(bar(kBarPEmpty), (u - 1) & 1u);
+    __syncwarp();
+  }
+
+  // ---------------------------------- exit ----------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (leader && warp == kWarpProducer && lane == 0 && *abort_flag) {
+    // After an abort, complete on behalf of the CTA that stopped first the fills the other one
+    // issued, and wait for every copy still in flight into either CTA (the follower's copies
+    // count their bytes here).  The two producers are at most one ring apart.
+    const uint32_t gf = *reinterpret_cast<volatile uint32_t*>(misc + kMiscPeerFills);
+    const uint32_t qf = *reinterpret_cast<volatile uint32_t*>(misc + kMiscPeerQ);
+    const uint32_t gmax = max(fills, gf);
+    for (uint32_t k = gmax > static_cast<uint32_t>(kNumSlots) ? gmax - kNumSlots : 0u; k < gmax; ++k) {
+      const uint32_t s = k % kNumSlots;
+      if (k >= fills) mbar_arrive(bar(kBarSlotFull + s));
+      if (k >= gf) mbar_arrive(bar(kBarSlotFull + s));
+      drain_wait(bar(kBarSlotFull + s), (k / kNumSlots) & 1u);
+    }
+    const uint32_t ql = static_cast<uint32_t>(q_fills);
+    const uint32_t qmax = max(ql, qf);
+    if (qmax > 0) {
+      const uint32_t k = qmax - 1;
+      if (k >= ql) mbar_arrive(bar(kBarQFull));
+      if (k >= qf) mbar_arrive(bar(kBarQFull));
+      drain_wait(bar(kBarQFull), k & 1u);
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
+                            cudaStream_t stream) {
+  auto kern = mla_decode_pair_kernel;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * p.num_sm_parts, p.row_groups, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_kv, p);
+  return static_cast<int>(e);
+}
+
+}  // namespace mla

@@ -28,8 +28,9 @@ part can be the continuation of a request started earlier.  Every block lands in
 exactly one chunk by construction.  Everything is a closed form of prefix sums, so the
 GPU kernel computes it in parallel.
 
-num_sm_parts: a CTA handles at most 64 query rows, so rows_per_kv_head rows need
-G = ceil(rows / 64) CTAs per chunk and num_sm_parts = max(1, sm_count // (h_kv * G)).
+num_sm_parts: up to 64 query rows run on one SM; more rows run on pairs of SMs that each
+carry 128 rows, so a chunk needs G = 1 SM (rows <= 64) or G = 2 * ceil(rows / 128) SMs, and
+num_sm_parts = max(1, sm_count // (h_kv * G)).
 """
 from __future__ import annotations
 
@@ -45,8 +46,16 @@ def row_groups_for(rows_per_kv_head: int) -> int:
     return max(1, (int(rows_per_kv_head) + ROWS_PER_CTA - 1) // ROWS_PER_CTA)
 
 
+PAIR_ROWS = 128
+
+
+def sms_per_part(rows_per_kv_head: int) -> int:
+    rows = int(rows_per_kv_head)
+    return 1 if rows <= ROWS_PER_CTA else 2 * ((rows + PAIR_ROWS - 1) // PAIR_ROWS)
+
+
 def num_sm_parts_for(rows_per_kv_head: int, h_kv: int, sm_count: int) -> int:
-    return max(1, int(sm_count) // (int(h_kv) * row_groups_for(rows_per_kv_head)))
+    return max(1, int(sm_count) // (int(h_kv) * sms_per_part(rows_per_kv_head)))
 
 
 def _blocks(L: int) -> int:

@@ -59,6 +59,9 @@ CASES = [
     ("r256_causal", 3, 2, 128, [2, 129, 1500], True),
     ("r48_pad_groups", 2, 1, 48, [257, 1], False),
     ("r96_two_groups", 2, 1, 96, [700, 128], False),
+    # CTA-pair path (more than 64 rows): odd block counts per chunk, a half-empty second pair
+    ("r128_odd_blocks", 4, 1, 128, [129, 385, 640, 1], False),
+    ("r192_two_pairs_causal", 2, 2, 96, [1000, 300], True),
 ]
 
 
@@ -110,6 +113,34 @@ def test_nan_in_unreadable_slots_does_not_leak():
     o2, l2, _, _ = run_gpu(dirty)
     assert np.isfinite(o2).all()
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_pair_fully_masked_rows_and_nan_tails():
+    # more than 64 rows (CTA pairs): causal rows that see nothing, an empty request, and NaN
+    # in every cache slot no request position covers
+    clean = mi.make_case(3, 3, 64, [1, 0, 200], causal=True, seed=26, poison=False, spare_blocks=4)
+    dirty = mi.make_case(3, 3, 64, [1, 0, 200], causal=True, seed=26, poison=True, spare_blocks=4)
+    O_ref, L_ref = oracle.mla_decode_reference(clean)
+    o1, l1, s1, _ = run_gpu(clean)
+    o2, l2, s2, _ = run_gpu(dirty)
+    assert s1 == 0 and s2 == 0
+    compare(clean, o1, l1, O_ref, L_ref)
+    assert np.isfinite(o2).all()
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_pair_block_table_permutation_is_bit_invariant():
+    case = mi.make_case(2, 1, 128, [700, 77], seed=27)
+    out1, lse1, _, _ = run_gpu(case)
+    rng = np.random.default_rng(6)
+    perm = rng.permutation(case.num_blocks)
+    kv2 = np.empty_like(case.kv)
+    kv2[perm] = case.kv
+    bt2 = case.block_table.copy()
+    bt2[bt2 >= 0] = perm[bt2[bt2 >= 0]]
+    case2 = mi.DecodeCase(**{**case.__dict__, "kv": kv2, "block_table": bt2})
+    out2, lse2, _, _ = run_gpu(case2)
+    assert np.array_equal(out1, out2) and np.array_equal(lse1, lse2)
 
 
 def test_split_count_invariance():

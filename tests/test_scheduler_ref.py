@@ -88,6 +88,9 @@ def test_num_sm_parts_rule():
     assert ts.num_sm_parts_for(128, 1, 148) == 74
     assert ts.num_sm_parts_for(256, 1, 148) == 37
     assert ts.num_sm_parts_for(256, 1, 2) == 1
+    assert ts.num_sm_parts_for(65, 1, 148) == 74      # one SM pair
+    assert ts.num_sm_parts_for(192, 1, 148) == 37     # two SM pairs
+    assert ts.num_sm_parts_for(300, 1, 148) == 24     # three SM pairs
 
 
 def test_planted_floor_division_is_caught():
