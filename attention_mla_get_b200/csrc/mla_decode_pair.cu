@@ -32,7 +32,7 @@
 // Ring: 16 KB slots (K slot = 128 tokens x 64 dims, V slot = one page x 128 dims).  Order per
 // chunk of n pair steps: K(0), K(1), then V(t), K(t + 2) for t = 0 .. n-1 (QK runs one step
 // ahead of PV).  Tokens past the request or the chunk are masked in S^T; their V rows (stale
-// ring contents or the cache's unused page tail) are zeroed by the leader before PV reads them.
+// ring contents or the cache's unused page tail) are zeroed by each CTA before PV reads them.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -76,8 +76,9 @@ static_assert(kOffP % 1024 == 0 && kOffSlots % 1024 == 0, "swizzle atoms need 10
 enum : int {
   kBarSlotFull = 0,                      // [kNumSlots] leader: both producers, count 2 + bytes
   kBarSlotEmpty = kBarSlotFull + kNumSlots,   // [kNumSlots] both: pair commit
-  kBarZFull = kBarSlotEmpty + kNumSlots,      // [kNumSlots] leader: V rows of a tail step zeroed
-  kBarSFull = kBarZFull + kNumSlots,          // [2] both: pair commit
+  kBarZFull = kBarSlotEmpty + kNumSlots,      // [kNumSlots] leader: both CTAs zeroed a tail V slot
+  kBarZLocal = kBarZFull + kNumSlots,         // [kNumSlots] both: this CTA's bytes of a tail V slot
+  kBarSFull = kBarZLocal + kNumSlots,         // [2] both: pair commit
   kBarSEmpty = kBarSFull + 2,                 // [2] leader: 16 softmax warps of the pair
   kBarPFull = kBarSEmpty + 2,                 // leader: the 8 warps that write P^T locally
   kBarPEmpty = kBarPFull + 1,                 // both: pair commit
@@ -256,7 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kNumSlots; ++i) {
       mbar_init(bar(kBarSlotFull + i), 2);
       mbar_init(bar(kBarSlotEmpty + i), 1);
-      mbar_init(bar(kBarZFull + i), 4);
+      mbar_init(bar(kBarZFull + i), 8);
+      mbar_init(bar(kBarZLocal + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
@@ -306,19 +308,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_rope = p.row_groups > 1 ? pol_keep : pol_stream;
       int last_use[kNumSlots];
       for (int i = 0; i < kNumSlots; ++i) last_use[i] = -1;
+      uint32_t zl_uses = 0, zl_par = 0;  // slots with a tail fill; parity of their last one
       bool ok = true;
       ChunkWalk walk(p, part);
       int b, c0, c1, split;
-      // two 64x64 boxes into one slot: (x0, y0) at +0 and (x1, y1) at +8 KB, each only if valid
-      auto fill = [&](int x0, int y0, bool v0, int x1, int y1, bool v1, uint64_t pol) -> bool {
+      // Two 64x64 boxes into one slot: (x0, y0) at +0 and (x1, y1) at +8 KB, each only if valid.
+      // The bytes count on the leader's full barrier, except for the V slots of a tail step: there
+      // they count on this CTA's own barrier, so that this CTA can zero the rows of tokens outside
+      // the request once its copy has landed (its softmax warps then arrive on the leader's ZFull).
+      auto fill = [&](int x0, int y0, bool v0, int x1, int y1, bool v1, uint64_t pol, bool tail) -> bool {
         const int s = static_cast<int>(fills % kNumSlots);
         const uint32_t use = fills / kNumSlots;
         if (!pwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
         const uint32_t full = lead(bar(kBarSlotFull + s));
-        mbar_arrive_expect_tx_relaxed(full, static_cast<uint32_t>(((v0 ? 1 : 0) + (v1 ? 1 : 0)) * kBoxBytes));
+        const uint32_t bytes = static_cast<uint32_t>(((v0 ? 1 : 0) + (v1 ? 1 : 0)) * kBoxBytes);
+        uint32_t dbar = full;
+        if (tail) {
+          mbar_arrive_expect_tx_relaxed(full, 0u);
+          mbar_arrive_expect_tx(bar(kBarZLocal + s), bytes);
+          dbar = map_to_cta(bar(kBarZLocal + s), rank);
+          zl_uses |= 1u << s;
+          zl_par ^= 1u << s;
+        } else {
+          mbar_arrive_expect_tx_relaxed(full, bytes);
+        }
         const uint32_t dst = sSlots + static_cast<uint32_t>(s) * kSlotBytes;
-        if (v0) tma_load_2d_pair(dst, &tm_kv, x0, y0, full, pol);
-        if (v1) tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x1, y1, full, pol);
+        if (v0) tma_load_2d_pair(dst, &tm_kv, x0, y0, dbar, pol);
+        if (v1) tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x1, y1, dbar, pol);
         last_use[s] = static_cast<int>(use);
         ++fills;
         return true;
@@ -347,17 +363,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ya = va ? bt[2 * kb] * kPage : 0;
             const int yb = vb ? bt[2 * kb + 1] * kPage : 0;
             for (int j = 0; ok && j < kKFills; ++j)
-              ok = fill(64 * j, ya, va, 64 * j, yb, vb, j < 8 ? pol_keep : pol_rope);
+              ok = fill(64 * j, ya, va, 64 * j, yb, vb, j < 8 ? pol_keep : pol_rope, false);
           } else {
             // V(t): this CTA's 256 output dims of all four pages of the step
+            const bool tail = is_tail(c0, c1, t, L);
+            bool v[4];
+            int y[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int pg = 2 * (c0 + 2 * t) + q;
+              v[q] = (c0 + 2 * t + (q >> 1) < c1) && pg < npages;
+              y[q] = v[q] ? bt[pg] * kPage : 0;
+            }
             for (int m = 0; ok && m < 2; ++m) {
               const int d = 256 * m + 128 * static_cast<int>(rank);
-              for (int q = 0; ok && q < 4; ++q) {
-                const int pg = 2 * (c0 + 2 * t) + q;
-                const bool v = (c0 + 2 * t + (q >> 1) < c1) && pg < npages;
-                const int y = v ? bt[pg] * kPage : 0;
-                ok = fill(d, y, v, d + 64, y, v, pol_v);
-              }
+              for (int q = 0; ok && q < 4; ++q) ok = fill(d, y[q], v[q], d + 64, y[q], v[q], pol_v, tail);
             }
           }
         }
@@ -367,6 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kNumSlots; ++s)
           if (last_use[s] >= 0) drain_wait(bar(kBarSlotEmpty + s), static_cast<uint32_t>(last_use[s]) & 1u);
         if (q_fills > 0) drain_wait(bar(kBarQEmpty), static_cast<uint32_t>(q_fills - 1) & 1u);
+      } else {
+        // copies of tail V slots count on this CTA's own barriers: let them land
+        for (int s = 0; s < kNumSlots; ++s)
+          if ((zl_uses >> s) & 1u) drain_wait(bar(kBarZLocal + s), ((zl_par >> s) & 1u) ^ 1u);
       }
       if (!leader) {
         st_cluster_u32(lead(sMisc + kMiscPeerFills), fills);
@@ -470,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float lsum[2] = {0.f, 0.f};
     uint32_t u = 0;
     uint32_t gchunk = 0;
+    uint32_t zlpar = 0;  // parity of each slot's next ZLocal phase
     int chunk = 0;
     bool fail = false;
     const int R = p.rows;
@@ -596,27 +621,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ok &= __shfl_sync(0xffffffffu, okp, 0) != 0;
         }
-        if (leader && tid < kRows && is_tail(c0, c1, t, L)) {
-          // zero, in both CTAs' V slots of this step, the rows of tokens outside the request or
-          // the chunk (the leader's full barrier counts both CTAs' bytes)
+        if (tid < kRows && is_tail(c0, c1, t, L)) {
+          // Zero, in this CTA's V slots of the step, the rows of tokens outside the request or the
+          // chunk (stale ring contents or the cache's unused page tail: 0 * NaN would poison O^T).
+          // These slots count their bytes on this CTA's own barrier; both CTAs then arrive on the
+          // leader's ZFull, which the MMA waits for before it reads the slot.
           const int r = tid & 63, box = tid >> 6;
           for (int k = 0; k < kVFills; ++k) {
             const uint32_t gv = gchunk + fills_before_v(t, n) + static_cast<uint32_t>(k);
             const uint32_t s = gv % kNumSlots;
-            ok &= warp_pwait(bar(kBarSlotFull + s), (gv / kNumSlots) & 1u, wc, lane);
+            ok &= warp_pwait(bar(kBarZLocal + s), (zlpar >> s) & 1u, wc, lane);
+            zlpar ^= 1u << s;
             const int q = k & 3;
             const int jj = (c0 + 2 * t) * kBlockTokens + 64 * q + r;
             if ((c0 + 2 * t + (q >> 1) >= c1) || jj >= L) {
               const uint32_t row = sSlots + s * kSlotBytes + static_cast<uint32_t>(box * kBoxBytes + r * 128);
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                st_shared_v4(row + 16u * c, 0u, 0u, 0u, 0u);
-                st_cluster_v4(other(row + 16u * c), 0u, 0u, 0u, 0u);
-              }
+              for (int c = 0; c < 8; ++c) st_shared_v4(row + 16u * c, 0u, 0u, 0u, 0u);
             }
-            fence_proxy_async_cluster();
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(lead(bar(kBarZFull + s)));
+            if (lane == 0) mbar_arrive_remote(lead(bar(kBarZFull + s)));
           }
         }
         fail |= !ok;
