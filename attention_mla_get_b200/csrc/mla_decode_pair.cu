@@ -51,17 +51,22 @@ constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
 constexpr int kRows = 128;        // query rows per pair
 constexpr int kHalfRows = 64;     // query rows of Q^T / P^T held by each CTA
-constexpr int kNumSlots = 7;
-constexpr int kSlotBytes = 16384;
-constexpr int kBoxBytes = 8192;   // 64 tokens x 64 dims bf16
-constexpr int kKFills = 9;        // K slots per step (576 dims / 64)
-constexpr int kVFills = 8;        // V slots per step (2 dim blocks x 4 pages)
+// The ring holds 32 KB stages of 8 MMAs each: every wait on a barrier in the MMA issue stream
+// idles the tensor pipe for ~200 cycles, so stages must carry enough MMA work to amortise it.
+constexpr int kNumSlots = 3;       // stages
+constexpr int kSlotBytes = 32768;
+constexpr int kHalfBytes = 16384;  // half a stage: 128 tokens x 64 dims, or one page x 128 dims
+constexpr int kRopeBytes = 16384;  // the 64 RoPE dims of a K step: a ring of its own (one slot)
+constexpr int kBoxBytes = 8192;    // 64 tokens x 64 dims bf16
+constexpr int kKFills = 4;         // K stages per step (dims 0-511 in 128-dim blocks)
+constexpr int kVFills = 4;         // V stages per step (2 dim blocks x 2 token blocks)
 constexpr int kQBytes = 9 * kBoxBytes;          // 64 rows x 576 dims
 constexpr int kPBytes = 256 * kHalfRows * 2;    // 256 tokens x 64 rows bf16
 constexpr int kOffQ = 0;
 constexpr int kOffP = kOffQ + kQBytes;
 constexpr int kOffSlots = kOffP + kPBytes;
-constexpr int kOffMisc = kOffSlots + kNumSlots * kSlotBytes;
+constexpr int kOffRope = kOffSlots + kNumSlots * kSlotBytes;
+constexpr int kOffMisc = kOffRope + kRopeBytes;
 constexpr int kMiscBytes = 6144;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 constexpr int kTmemCols = 512;
@@ -70,7 +75,8 @@ constexpr int kColS = 256;    // S^T buffer sb at columns 256 + 128 sb
 constexpr uint32_t kIdescQK = idesc_bf16(256, kRows, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16(256, kRows, true, true);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kOffP % 1024 == 0 && kOffSlots % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+static_assert(kOffP % 1024 == 0 && kOffSlots % 1024 == 0 && kOffRope % 1024 == 0,
+              "swizzle atoms need 1024-byte alignment");
 
 // misc area: barriers, then scalars, then per-row scratch
 enum : int {
@@ -78,7 +84,9 @@ enum : int {
   kBarSlotEmpty = kBarSlotFull + kNumSlots,   // [kNumSlots] both: pair commit
   kBarZFull = kBarSlotEmpty + kNumSlots,      // [kNumSlots] leader: both CTAs zeroed a tail V slot
   kBarZLocal = kBarZFull + kNumSlots,         // [kNumSlots] both: this CTA's bytes of a tail V slot
-  kBarSFull = kBarZLocal + kNumSlots,         // [2] both: pair commit
+  kBarRopeFull = kBarZLocal + kNumSlots,      // leader: both producers, count 2 + bytes
+  kBarRopeEmpty = kBarRopeFull + 1,           // both: pair commit
+  kBarSFull = kBarRopeEmpty + 1,              // [2] both: pair commit
   kBarSEmpty = kBarSFull + 2,                 // [2] leader: 16 softmax warps of the pair
   kBarPFull = kBarSEmpty + 2,                 // leader: the 8 warps that write P^T locally
   kBarPEmpty = kBarPFull + 1,                 // both: pair commit
@@ -96,6 +104,7 @@ constexpr int kMiscHolder = 512;   // TMEM base address
 constexpr int kMiscAbort = 516;    // abort flag
 constexpr int kMiscPeerFills = 520;// follower's slot fills (written into the leader at exit)
 constexpr int kMiscPeerQ = 524;    // follower's Q fills
+constexpr int kMiscPeerRope = 528; // follower's RoPE fills
 constexpr int kMiscRed = 1024;     // float [4 lane quadrants][128 rows]
 constexpr int kMiscM = 3072;       // float [128]
 constexpr int kMiscAlpha = 3584;   // float [128]
@@ -161,8 +170,8 @@ __device__ __forceinline__ bool is_tail(int c0, int c1, int t, int L) {
   return (c0 + 2 * t + 1 >= c1) || ((c0 + 2 * t + 2) * kBlockTokens > L);
 }
 
-// Bounded waits (cluster-scope acquire).  On time-out: status bit, this CTA's and the peer's
-// abort flags; every waiter of both CTAs then unwinds.
+// Bounded waits.  On time-out: status bit, this CTA's and the peer's abort flags; every waiter
+// of both CTAs then unwinds.
 struct PairCtl {
   volatile int* abort_flag;
   uint32_t peer_abort;  // cluster address of the peer's abort flag
@@ -177,10 +186,10 @@ static __device__ __noinline__ void pair_timeout(const PairCtl& c) {
 }
 
 __device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, const PairCtl& c) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (*c.abort_flag) return false;
     if (clock64() - t0 > kWaitLimitCycles) {
       pair_timeout(c);
@@ -192,7 +201,7 @@ __device__ __forceinline__ bool pwait(uint32_t bar, uint32_t parity, const PairC
 // used only at exit: bounded, ignores the abort flag
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
-  while (!mbar_try_wait_cluster(bar, parity)) {
+  while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > kWaitLimitCycles) return;
   }
 }
@@ -229,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = sbase + kOffQ;
   const uint32_t sP = sbase + kOffP;
   const uint32_t sSlots = sbase + kOffSlots;
+  const uint32_t sRope = sbase + kOffRope;
   uint8_t* misc = smem + kOffMisc;
   const uint32_t sMisc = smem_u32(misc);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + kMiscHolder);
@@ -260,6 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarZFull + i), 8);
       mbar_init(bar(kBarZLocal + i), 1);
     }
+    mbar_init(bar(kBarRopeFull), 2);
+    mbar_init(bar(kBarRopeEmpty), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarSEmpty + i), 16);
@@ -277,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerFills) = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerQ) = 0;
+    *reinterpret_cast<uint32_t*>(misc + kMiscPeerRope) = 0;
     fence_barrier_init();
   }
   if (warp == kWarpProducer && lane == 0) {
@@ -296,8 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
 
   // state the exit sequence needs
-  uint32_t fills = 0;  // producer: slot fills issued
+  uint32_t fills = 0;  // producer: stage fills issued
   int q_fills = 0;     // producer: Q fills issued
+  int rope_fills = 0;  // producer: RoPE slot fills issued
 
   if (warp == kWarpProducer) {
     // ================================ TMA producer ================================
@@ -312,16 +326,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       ChunkWalk walk(p, part);
       int b, c0, c1, split;
-      // Two 64x64 boxes into one slot: (x0, y0) at +0 and (x1, y1) at +8 KB, each only if valid.
-      // The bytes count on the leader's full barrier, except for the V slots of a tail step: there
-      // they count on this CTA's own barrier, so that this CTA can zero the rows of tokens outside
-      // the request once its copy has landed (its softmax warps then arrive on the leader's ZFull).
-      auto fill = [&](int x0, int y0, bool v0, int x1, int y1, bool v1, uint64_t pol, bool tail) -> bool {
+      // One stage = four 64x64 boxes: box (x[i], y[i]) lands at +8 KB * i and is copied only if
+      // valid[i] (a page of the request).  The bytes count on the leader's full barrier, except for the
+      // V stages of a tail step: there they count on this CTA's own barrier, so that this CTA can
+      // zero the rows of tokens outside the request once its copy has landed (its softmax warps
+      // then arrive on the leader's ZFull).
+      auto fill = [&](const int* x, const int* y, const bool* valid, uint64_t pol, bool tail) -> bool {
         const int s = static_cast<int>(fills % kNumSlots);
         const uint32_t use = fills / kNumSlots;
         if (!pwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
         const uint32_t full = lead(bar(kBarSlotFull + s));
-        const uint32_t bytes = static_cast<uint32_t>(((v0 ? 1 : 0) + (v1 ? 1 : 0)) * kBoxBytes);
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bytes += valid[i] ? static_cast<uint32_t>(kBoxBytes) : 0u;
         uint32_t dbar = full;
         if (tail) {
           mbar_arrive_expect_tx_relaxed(full, 0u);
@@ -333,8 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx_relaxed(full, bytes);
         }
         const uint32_t dst = sSlots + static_cast<uint32_t>(s) * kSlotBytes;
-        if (v0) tma_load_2d_pair(dst, &tm_kv, x0, y0, dbar, pol);
-        if (v1) tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x1, y1, dbar, pol);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (valid[i]) tma_load_2d_pair(dst + i * kBoxBytes, &tm_kv, x[i], y[i], dbar, pol);
         last_use[s] = static_cast<int>(use);
         ++fills;
         return true;
@@ -356,16 +374,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           int t;
           order_at(e, n, is_v, t);
           if (!is_v) {
-            // K(t): this CTA's own 128-token block, all 576 dims
+            // K(t): this CTA's own 128-token block (pages a, b), all 576 dims
             const int kb = c0 + 2 * t + static_cast<int>(rank);
             const bool va = kb < c1;
             const bool vb = va && (2 * kb + 1 < npages);
             const int ya = va ? bt[2 * kb] * kPage : 0;
             const int yb = vb ? bt[2 * kb + 1] * kPage : 0;
-            for (int j = 0; ok && j < kKFills; ++j)
-              ok = fill(64 * j, ya, va, 64 * j, yb, vb, j < 8 ? pol_keep : pol_rope, false);
+            {
+              // the RoPE dims first: QK(t) starts with them
+              const uint32_t use = static_cast<uint32_t>(rope_fills);
+              if (!pwait(bar(kBarRopeEmpty), (use & 1u) ^ 1u, wc)) { ok = false; break; }
+              const uint32_t rfull = lead(bar(kBarRopeFull));
+              mbar_arrive_expect_tx_relaxed(rfull, static_cast<uint32_t>(((va ? 1 : 0) + (vb ? 1 : 0)) * kBoxBytes));
+              if (va) tma_load_2d_pair(sRope, &tm_kv, kDv, ya, rfull, pol_rope);
+              if (vb) tma_load_2d_pair(sRope + kBoxBytes, &tm_kv, kDv, yb, rfull, pol_rope);
+              ++rope_fills;
+            }
+            for (int j = 0; ok && j < kKFills; ++j) {
+              // half h = dims 128j + 64h .. +63 of both pages (page a at +0, page b at +8 KB)
+              const int x[4] = {128 * j, 128 * j, 128 * j + 64, 128 * j + 64};
+              const int yy[4] = {ya, yb, ya, yb};
+              const bool vv[4] = {va, vb, va, vb};
+              ok = fill(x, yy, vv, pol_keep, false);
+            }
           } else {
-            // V(t): this CTA's 256 output dims of all four pages of the step
+            // V(t): this CTA's 256 output dims of the step's two token blocks; stage (m, blk) holds
+            // dims 256m + 128 rank .. +127 of pages 2(c0 + 2t + blk) (+0) and +1 (+16 KB)
             const bool tail = is_tail(c0, c1, t, L);
             bool v[4];
             int y[4];
@@ -377,7 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int m = 0; ok && m < 2; ++m) {
               const int d = 256 * m + 128 * static_cast<int>(rank);
-              for (int q = 0; ok && q < 4; ++q) ok = fill(d, y[q], v[q], d + 64, y[q], v[q], pol_v, tail);
+              for (int blk = 0; ok && blk < 2; ++blk) {
+                const int x[4] = {d, d + 64, d, d + 64};
+                const int yy[4] = {y[2 * blk], y[2 * blk], y[2 * blk + 1], y[2 * blk + 1]};
+                const bool vv[4] = {v[2 * blk], v[2 * blk], v[2 * blk + 1], v[2 * blk + 1]};
+                ok = fill(x, yy, vv, pol_v, tail);
+              }
             }
           }
         }
@@ -387,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kNumSlots; ++s)
           if (last_use[s] >= 0) drain_wait(bar(kBarSlotEmpty + s), static_cast<uint32_t>(last_use[s]) & 1u);
         if (q_fills > 0) drain_wait(bar(kBarQEmpty), static_cast<uint32_t>(q_fills - 1) & 1u);
+        if (rope_fills > 0) drain_wait(bar(kBarRopeEmpty), static_cast<uint32_t>(rope_fills - 1) & 1u);
       } else {
         // copies of tail V slots count on this CTA's own barriers: let them land
         for (int s = 0; s < kNumSlots; ++s)
@@ -395,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!leader) {
         st_cluster_u32(lead(sMisc + kMiscPeerFills), fills);
         st_cluster_u32(lead(sMisc + kMiscPeerQ), static_cast<uint32_t>(q_fills));
+        st_cluster_u32(lead(sMisc + kMiscPeerRope), static_cast<uint32_t>(rope_fills));
       }
     }
   } else if (warp == kWarpMma) {
@@ -403,6 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0;   // slot fills consumed
       uint32_t u = 0;   // QK steps issued
       uint32_t up = 0;  // PV steps issued
+      uint32_t rope_used = 0;
       uint32_t zpar = 0;
       int chunk = 0;
       bool ok = true;
@@ -412,7 +454,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         s = g % kNumSlots;
         if (!pwait(bar(kBarSlotFull + s), (g / kNumSlots) & 1u, wc)) return false;
         ++g;
-        tc_fence_after();
         return true;
       };
       while (ok && walk.next(p, b, c0, c1, split)) {
@@ -425,18 +466,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           order_at(e, n, is_v, t);
           if (!is_v) {
             const int sb = static_cast<int>(u & 1u);
+            // the softmax warps finished their tcgen05.ld of this buffer (wait::ld) before arriving
             if (!pwait(bar(kBarSEmpty + sb), ((u >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
-            tc_fence_after();
             const uint32_t d = tmem + kColS + 128u * sb;
+            // RoPE dims first (they have their own slot), then the four 128-dim K stages
+            if (!pwait(bar(kBarRopeFull), rope_used & 1u, wc)) { ok = false; break; }
+            ++rope_used;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_pair(d, smem_desc(sRope + 32 * kk, 16, 1024, kSwizzle128),
+                             smem_desc(sQ + 8 * kBoxBytes + 32 * kk, 16, 1024, kSwizzle128), kIdescQK,
+                             kk != 0 ? 1u : 0u);
+            umma_commit_pair_mc(bar(kBarRopeEmpty), 0x3);
             for (int j = 0; ok && j < kKFills; ++j) {
               uint32_t s;
               if (!next_slot(s)) { ok = false; break; }
               const uint32_t kbase = sSlots + s * kSlotBytes;
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                umma_bf16_pair(d, smem_desc(kbase + 32 * kk, 16, 1024, kSwizzle128),
-                               smem_desc(sQ + j * kBoxBytes + 32 * kk, 16, 1024, kSwizzle128), kIdescQK,
-                               (j | kk) != 0 ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk)
+                umma_bf16_pair(d, smem_desc(kbase + (kk >> 2) * kHalfBytes + 32 * (kk & 3), 16, 1024, kSwizzle128),
+                               smem_desc(sQ + (2 * j + (kk >> 2)) * kBoxBytes + 32 * (kk & 3), 16, 1024, kSwizzle128),
+                               kIdescQK, 1u);
               umma_commit_pair_mc(bar(kBarSlotEmpty + s), 0x3);
             }
             if (!ok) break;
@@ -446,23 +496,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             if (!pwait(bar(kBarPFull), up & 1u, wc)) { ok = false; break; }
             if (t == 0 && !pwait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) { ok = false; break; }
+            // orders PV after the softmax warps' rescale of O^T (tcgen05.st) -- once per step: a
+            // tcgen05 fence in the issue stream drains the MMA pipe, so none sits before
+            // operands that only TMA or shared-memory stores produced
             tc_fence_after();
             const bool tail = is_tail(c0, c1, t, L);
             for (int m = 0; ok && m < 2; ++m) {
-              for (int q = 0; q < 4; ++q) {
+              for (int blk = 0; blk < 2; ++blk) {
                 uint32_t s;
                 if (!next_slot(s)) { ok = false; break; }
                 if (tail) {
                   if (!pwait(bar(kBarZFull + s), (zpar >> s) & 1u, wc)) { ok = false; break; }
                   zpar ^= 1u << s;
-                  tc_fence_after();
                 }
                 const uint32_t vbase = sSlots + s * kSlotBytes;
+                // half h = page 2 blk + h of the step (64 tokens x 128 dims, 64-dim boxes 8 KB apart)
 #pragma unroll
-                for (int kt = 0; kt < 4; ++kt)
-                  umma_bf16_pair(tmem + kColO + 128u * m, smem_desc(vbase + 2048 * kt, kBoxBytes, 1024, kSwizzle128),
-                                 smem_desc(sP + (64 * q + 16 * kt) * 128, kBoxBytes, 1024, kSwizzle128), kIdescPV,
-                                 (t == 0 && q == 0 && kt == 0) ? 0u : 1u);
+                for (int kt = 0; kt < 8; ++kt)
+                  umma_bf16_pair(tmem + kColO + 128u * m,
+                                 smem_desc(vbase + (kt >> 2) * kHalfBytes + 2048 * (kt & 3), kBoxBytes, 1024, kSwizzle128),
+                                 smem_desc(sP + (128 * blk + 16 * kt) * 128, kBoxBytes, 1024, kSwizzle128), kIdescPV,
+                                 (t == 0 && blk == 0 && kt == 0) ? 0u : 1u);
                 umma_commit_pair_mc(bar(kBarSlotEmpty + s), 0x3);
               }
             }
@@ -626,18 +680,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           // chunk (stale ring contents or the cache's unused page tail: 0 * NaN would poison O^T).
           // These slots count their bytes on this CTA's own barrier; both CTAs then arrive on the
           // leader's ZFull, which the MMA waits for before it reads the slot.
-          const int r = tid & 63, box = tid >> 6;
+          const int r = tid & 63, h = tid >> 6;  // row r of page h of the stage's token block
           for (int k = 0; k < kVFills; ++k) {
             const uint32_t gv = gchunk + fills_before_v(t, n) + static_cast<uint32_t>(k);
             const uint32_t s = gv % kNumSlots;
             ok &= warp_pwait(bar(kBarZLocal + s), (zlpar >> s) & 1u, wc, lane);
             zlpar ^= 1u << s;
-            const int q = k & 3;
-            const int jj = (c0 + 2 * t) * kBlockTokens + 64 * q + r;
-            if ((c0 + 2 * t + (q >> 1) >= c1) || jj >= L) {
-              const uint32_t row = sSlots + s * kSlotBytes + static_cast<uint32_t>(box * kBoxBytes + r * 128);
+            const int blk = k & 1;  // stages go (m = 0, blk 0), (0, 1), (1, 0), (1, 1)
+            const int jj = (c0 + 2 * t + blk) * kBlockTokens + 64 * h + r;
+            if ((c0 + 2 * t + blk >= c1) || jj >= L) {
+              const uint32_t row = sSlots + s * kSlotBytes + static_cast<uint32_t>(h * kHalfBytes + r * 128);
 #pragma unroll
-              for (int c = 0; c < 8; ++c) st_shared_v4(row + 16u * c, 0u, 0u, 0u, 0u);
+              for (int c = 0; c < 8; ++c) {
+                st_shared_v4(row + 16u * c, 0u, 0u, 0u, 0u);
+                st_shared_v4(row + kBoxBytes + 16u * c, 0u, 0u, 0u, 0u);
+              }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -730,6 +787,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (k >= ql) mbar_arrive(bar(kBarQFull));
       if (k >= qf) mbar_arrive(bar(kBarQFull));
       drain_wait(bar(kBarQFull), k & 1u);
+    }
+    const uint32_t rf = *reinterpret_cast<volatile uint32_t*>(misc + kMiscPeerRope);
+    const uint32_t rl = static_cast<uint32_t>(rope_fills);
+    const uint32_t rmax = max(rl, rf);
+    if (rmax > 0) {
+      const uint32_t k = rmax - 1;
+      if (k >= rl) mbar_arrive(bar(kBarRopeFull));
+      if (k >= rf) mbar_arrive(bar(kBarRopeFull));
+      drain_wait(bar(kBarRopeFull), k & 1u);
     }
   }
   __syncthreads();
