@@ -481,12 +481,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; ok && j < kKFills; ++j) {
               uint32_t s;
               if (!next_slot(s)) { ok = false; break; }
-              const uint32_t kbase = sSlots + s * kSlotBytes;
+              // descriptors advance by (byte offset >> 4) in their start-address field
+              const uint64_t a0 = smem_desc(sSlots + s * kSlotBytes, 16, 1024, kSwizzle128);
+              const uint64_t b0 = smem_desc(sQ + 2 * j * kBoxBytes, 16, 1024, kSwizzle128);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                umma_bf16_pair(d, smem_desc(kbase + (kk >> 2) * kHalfBytes + 32 * (kk & 3), 16, 1024, kSwizzle128),
-                               smem_desc(sQ + (2 * j + (kk >> 2)) * kBoxBytes + 32 * (kk & 3), 16, 1024, kSwizzle128),
-                               kIdescQK, 1u);
+                umma_bf16_pair(d, a0 + static_cast<uint64_t>(((kk >> 2) * kHalfBytes + 32 * (kk & 3)) >> 4),
+                               b0 + static_cast<uint64_t>(((kk >> 2) * kBoxBytes + 32 * (kk & 3)) >> 4), kIdescQK, 1u);
               umma_commit_pair_mc(bar(kBarSlotEmpty + s), 0x3);
             }
             if (!ok) break;
@@ -509,13 +510,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                   if (!pwait(bar(kBarZFull + s), (zpar >> s) & 1u, wc)) { ok = false; break; }
                   zpar ^= 1u << s;
                 }
-                const uint32_t vbase = sSlots + s * kSlotBytes;
                 // half h = page 2 blk + h of the step (64 tokens x 128 dims, 64-dim boxes 8 KB apart)
+                const uint64_t a0 = smem_desc(sSlots + s * kSlotBytes, kBoxBytes, 1024, kSwizzle128);
+                const uint64_t b0 = smem_desc(sP + 128 * blk * 128, kBoxBytes, 1024, kSwizzle128);
 #pragma unroll
                 for (int kt = 0; kt < 8; ++kt)
                   umma_bf16_pair(tmem + kColO + 128u * m,
-                                 smem_desc(vbase + (kt >> 2) * kHalfBytes + 2048 * (kt & 3), kBoxBytes, 1024, kSwizzle128),
-                                 smem_desc(sP + (128 * blk + 16 * kt) * 128, kBoxBytes, 1024, kSwizzle128), kIdescPV,
+                                 a0 + static_cast<uint64_t>(((kt >> 2) * kHalfBytes + 2048 * (kt & 3)) >> 4),
+                                 b0 + static_cast<uint64_t>((16 * kt * 128) >> 4), kIdescPV,
                                  (t == 0 && blk == 0 && kt == 0) ? 0u : 1u);
                 umma_commit_pair_mc(bar(kBarSlotEmpty + s), 0x3);
               }
@@ -733,14 +735,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       fail |= !ok;
       tc_fence_after();
       {
+        // O^T block h of this CTA: dim = lane's output dim, columns = query rows.  The tensor
+        // memory is released (OEmpty) as soon as the last load has landed, before its stores.
         const int dim = 256 * h + 128 * static_cast<int>(rank) + tl;
 #pragma unroll
-        for (int c = 0; c < kRows; c += 16) {
-          float o[16];
+        for (int c = 0; c < kRows; c += 32) {
+          float o[32];
           tmem_ld16(tmem + lane_base + kColO + 128u * h + c, o);
+          tmem_ld16(tmem + lane_base + kColO + 128u * h + c + 16, o + 16);
           tmem_wait_ld();
+          if (c + 32 == kRows) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(lead(bar(kBarOEmpty)));
+          }
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
+          for (int e = 0; e < 32; ++e) {
             const int row = row0 + c + e;
             if (row < R) {
               const float val = o[e] * inv_sm[c + e];
@@ -752,9 +762,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead(bar(kBarOEmpty)));
       gchunk += static_cast<uint32_t>(kKFills + kVFills) * static_cast<uint32_t>(n);
       ++chunk;
     }
