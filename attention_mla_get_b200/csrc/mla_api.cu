@@ -194,9 +194,10 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = pair                      ? mla::launch_decode_pair_bf16(tm_q, tm_kv, p, st)
-          : kv_dtype == MLA_KV_BF16 ? mla::launch_decode_bf16(tm_q, tm_kv, p, rg, st)
-                                    : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, rg, st);
+  int e = kv_dtype == MLA_KV_BF16 ? (pair ? mla::launch_decode_pair_bf16(tm_q, tm_kv, p, st)
+                                          : mla::launch_decode_bf16(tm_q, tm_kv, p, rg, st))
+          : pair ? mla::launch_decode_pair_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, st)
+                 : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
 
   mla::CombineParams cp{};

@@ -29,11 +29,22 @@
 // CTA writes the bf16 P^T rows of its tokens into both CTAs' P^T halves (64 query rows each).
 // Row sums are exchanged once per chunk.
 //
-// Ring: 16 KB slots (K slot = 128 tokens x 64 dims, V slot = one page x 128 dims).  Order per
-// chunk of n pair steps: K(0), K(1), then V(t), K(t + 2) for t = 0 .. n-1 (QK runs one step
-// ahead of PV).  Tokens past the request or the chunk are masked in S^T; their V rows (stale
-// ring contents or the cache's unused page tail) are zeroed by each CTA before PV reads them.
+// Ring: 32 KB stages (K stage = 128 tokens x 128 dims, V stage = two pages x 128 dims) and a
+// separate slot for the 64 RoPE dims of a K step.  Order per chunk of n pair steps: K(0), K(1),
+// then V(t), K(t + 2) for t = 0 .. n-1 (QK runs one step ahead of PV).  Tokens past the request
+// or the chunk are masked in S^T; their V rows (stale ring contents or the cache's unused page
+// tail) are zeroed by each CTA before PV reads them.
+//
+// FP8 cache (656-byte tokens: 512 e4m3 codes, 4 fp32 scales per 128 dims, 64 bf16 RoPE dims;
+// the wmrh.cn page, "FP8 KV缓存内存效率" table): the producer TMA-loads raw code columns (128
+// dims x 2 pages) with their scales into a raw ring of this CTA; two dequant warps write each
+// stage of the same order as f16 (code * scale) into the 32 KB stages, with zeros for tokens
+// outside the request, and convert the Q tile and each RoPE slot from bf16 to f16 in place.
+// The MMAs then run on f16 operands: e4m3 codes are exact in f16, which also keeps 11
+// mantissa bits of q, P and code * scale where bf16 keeps 8 (f16's range, |x| < 65504, holds
+// for the scaled cache and the queries).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "mla_internal.h"
@@ -45,15 +56,16 @@ namespace {
 
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units
 constexpr float kLn2 = 0.69314718055994530942f;
-constexpr int kThreads = 320;     // warps 0-7 softmax + epilogue, 8 producer, 9 MMA / TMEM owner
+// warps 0-7 softmax + epilogue, 8 producer, 9 MMA issuer / TMEM owner, 10-13 FP8 dequant
 constexpr int kSoftmaxThreads = 256;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
+constexpr int kWarpDequant = 10;
+constexpr int kDequantThreads = 128;
 constexpr int kRows = 128;        // query rows per pair
 constexpr int kHalfRows = 64;     // query rows of Q^T / P^T held by each CTA
 // The ring holds 32 KB stages of 8 MMAs each: every wait on a barrier in the MMA issue stream
 // idles the tensor pipe for ~200 cycles, so stages must carry enough MMA work to amortise it.
-constexpr int kNumSlots = 3;       // stages
 constexpr int kSlotBytes = 32768;
 constexpr int kHalfBytes = 16384;  // half a stage: 128 tokens x 64 dims, or one page x 128 dims
 constexpr int kRopeBytes = 16384;  // the 64 RoPE dims of a K step: a ring of its own (one slot)
@@ -62,35 +74,57 @@ constexpr int kKFills = 4;         // K stages per step (dims 0-511 in 128-dim b
 constexpr int kVFills = 4;         // V stages per step (2 dim blocks x 2 token blocks)
 constexpr int kQBytes = 9 * kBoxBytes;          // 64 rows x 576 dims
 constexpr int kPBytes = 256 * kHalfRows * 2;    // 256 tokens x 64 rows bf16
+constexpr int kRawCodeBytes = 16384;  // FP8: 128 dims x 2 pages of e4m3 codes
+constexpr int kRawScaleBytes = 2048;  // FP8: the 4 fp32 scales of those 128 tokens
+constexpr int kRawBytes = kRawCodeBytes + kRawScaleBytes;
+constexpr int kNumRaw = 2;
 constexpr int kOffQ = 0;
 constexpr int kOffP = kOffQ + kQBytes;
 constexpr int kOffSlots = kOffP + kPBytes;
-constexpr int kOffRope = kOffSlots + kNumSlots * kSlotBytes;
-constexpr int kOffMisc = kOffRope + kRopeBytes;
 constexpr int kMiscBytes = 6144;
-constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 constexpr int kTmemCols = 512;
 constexpr int kColO = 0;      // O^T dim block m at columns 128m
 constexpr int kColS = 256;    // S^T buffer sb at columns 256 + 128 sb
-constexpr uint32_t kIdescQK = idesc_bf16(256, kRows, false, false);
-constexpr uint32_t kIdescPV = idesc_bf16(256, kRows, true, true);
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kOffP % 1024 == 0 && kOffSlots % 1024 == 0 && kOffRope % 1024 == 0,
-              "swizzle atoms need 1024-byte alignment");
+
+// f16 operands (FP8 cache): the A and B format fields of the instruction descriptor are 0
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16(M, N, a_mn_major, b_mn_major) & ~((7u << 7) | (7u << 10));
+}
+
+template <bool FP8>
+struct PairCfg {
+  // FP8: 16 warps (two idle) so that the compiler keeps every thread within 128 registers, the
+  // per-SM-sub-partition share of 4 resident warps
+  static constexpr int kThreads = FP8 ? 512 : 320;
+  static constexpr int kNumSlots = FP8 ? 2 : 3;  // FP8 gives a stage to the raw ring
+  static constexpr int kOffRaw = kOffSlots + kNumSlots * kSlotBytes;
+  static constexpr int kOffRope = kOffRaw + (FP8 ? kNumRaw * kRawBytes : 0);
+  static constexpr int kOffMisc = kOffRope + kRopeBytes;
+  static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kIdescQK = FP8 ? idesc_f16(256, kRows, false, false) : idesc_bf16(256, kRows, false, false);
+  static constexpr uint32_t kIdescPV = FP8 ? idesc_f16(256, kRows, true, true) : idesc_bf16(256, kRows, true, true);
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kOffSlots % 1024 == 0 && kOffRope % 1024 == 0 && kOffRaw % 128 == 0,
+                "swizzle atoms need 1024-byte alignment");
+};
+static_assert(kOffP % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+constexpr int kMaxSlots = 3;
 
 // misc area: barriers, then scalars, then per-row scratch
 enum : int {
-  kBarSlotFull = 0,                      // [kNumSlots] leader: both producers, count 2 + bytes
-  kBarSlotEmpty = kBarSlotFull + kNumSlots,   // [kNumSlots] both: pair commit
-  kBarZFull = kBarSlotEmpty + kNumSlots,      // [kNumSlots] leader: both CTAs zeroed a tail V slot
-  kBarZLocal = kBarZFull + kNumSlots,         // [kNumSlots] both: this CTA's bytes of a tail V slot
-  kBarRopeFull = kBarZLocal + kNumSlots,      // leader: both producers, count 2 + bytes
+  // [stages] leader: both producers (FP8: both dequant groups), count 2 + bytes
+  kBarSlotFull = 0,
+  kBarSlotEmpty = kBarSlotFull + kMaxSlots,   // [stages] both: pair commit
+  kBarZFull = kBarSlotEmpty + kMaxSlots,      // [stages] leader: both CTAs zeroed a tail V slot
+  kBarZLocal = kBarZFull + kMaxSlots,         // [stages] both: this CTA's bytes of a tail V slot
+  // leader: both producers, count 2 + bytes (FP8: this CTA's producer, count 1 + bytes)
+  kBarRopeFull = kBarZLocal + kMaxSlots,
   kBarRopeEmpty = kBarRopeFull + 1,           // both: pair commit
   kBarSFull = kBarRopeEmpty + 1,              // [2] both: pair commit
   kBarSEmpty = kBarSFull + 2,                 // [2] leader: 16 softmax warps of the pair
   kBarPFull = kBarSEmpty + 2,                 // leader: the 8 warps that write P^T locally
   kBarPEmpty = kBarPFull + 1,                 // both: pair commit
-  kBarQFull = kBarPEmpty + 1,                 // leader: both producers
+  kBarQFull = kBarPEmpty + 1,                 // leader: both producers (FP8: this CTA's, count 1)
   kBarQEmpty = kBarQFull + 1,                 // both: pair commit
   kBarOFull = kBarQEmpty + 1,                 // both: pair commit
   kBarOEmpty = kBarOFull + 1,                 // leader: 16 epilogue warps
@@ -98,7 +132,11 @@ enum : int {
   kBarMaxFull = kBarDrain + 1,                // [2] both: 512 bytes of the peer's block maxima
   kBarLFull = kBarMaxFull + 2,                // both: 512 bytes of the peer's row sums
   kBarPRecv = kBarLFull + 1,                  // both: 16 KB of P^T rows from the peer
-  kNumBars = kBarPRecv + 1,
+  kBarRawFull = kBarPRecv + 1,                // [2] FP8, both: this CTA's raw fill, count 1 + bytes
+  kBarRawEmpty = kBarRawFull + kNumRaw,       // [2] FP8, both: this CTA's dequant group
+  kBarQReady = kBarRawEmpty + kNumRaw,        // FP8, leader: Q in f16 in both CTAs, count 2
+  kBarRopeReady = kBarQReady + 1,             // FP8, leader: RoPE slot in f16 in both CTAs, count 2
+  kNumBars = kBarRopeReady + 1,
 };
 constexpr int kMiscHolder = 512;   // TMEM base address
 constexpr int kMiscAbort = 516;    // abort flag
@@ -229,17 +267,86 @@ __device__ __forceinline__ void reduce_scatter64_sum(float* v, int lane) {
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// bf16 pair -> f16 pair (round to nearest even)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// Two e4m3 codes (low 16 bits) -> f16 pair of code * scale.  The codes are exact in f16; with
+// the scale an f16 normal number (scale2 = that f16 twice) the product is one f16 multiply.
+__device__ __forceinline__ uint32_t e4m3x2_times_f16x2(uint32_t codes, uint32_t scale2) {
+  uint32_t h, r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(codes & 0xFFFFu)));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(scale2));
+  return r;
+}
+// The same with the product formed in fp32 (scales outside the f16 normal range).
+__device__ __forceinline__ uint32_t e4m3x2_times_f32(uint32_t codes, float scale) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(codes & 0xFFFFu)));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_f16x2(f.x * scale, f.y * scale);
+}
+
+// One token row of an FP8 stage: 128 e4m3 codes at `src` times `scale`, as f16 into the two
+// 64-dim halves of a swizzled stage row (`dst`, halves `hstride` apart; row index `row`).  All
+// eight 16-byte loads are issued before the first conversion, so their latencies overlap.
+__device__ __forceinline__ void dequant_row(uint32_t src, uint32_t dst, uint32_t hstride, uint32_t row, float scale) {
+  const uint32_t swz = row & 7u;
+  uint32_t w[8][4];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t cc = (static_cast<uint32_t>(c) + row) & 7u;  // spread the banks
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(w[c][0]), "=r"(w[c][1]), "=r"(w[c][2]), "=r"(w[c][3])
+                 : "r"(src + 16u * cc));
+  }
+  if (scale >= 6.103515625e-05f && scale <= 146.0f) {  // f16 normal scale, |448 scale| < 65504
+    const __half2 s2h = __float2half2_rn(scale);
+    const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&s2h);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t cc = (static_cast<uint32_t>(c) + row) & 7u;
+      // codes 16cc .. 16cc + 15: dim half cc / 4, 16-byte chunks 2 (cc % 4) and + 1
+      const uint32_t base = dst + (cc >> 2) * hstride;
+      const uint32_t q0 = 2u * (cc & 3u);
+      st_shared_v4(base + ((q0 ^ swz) << 4), e4m3x2_times_f16x2(w[c][0], s2), e4m3x2_times_f16x2(w[c][0] >> 16, s2),
+                   e4m3x2_times_f16x2(w[c][1], s2), e4m3x2_times_f16x2(w[c][1] >> 16, s2));
+      st_shared_v4(base + (((q0 + 1u) ^ swz) << 4), e4m3x2_times_f16x2(w[c][2], s2),
+                   e4m3x2_times_f16x2(w[c][2] >> 16, s2), e4m3x2_times_f16x2(w[c][3], s2),
+                   e4m3x2_times_f16x2(w[c][3] >> 16, s2));
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t cc = (static_cast<uint32_t>(c) + row) & 7u;
+      const uint32_t base = dst + (cc >> 2) * hstride;
+      const uint32_t q0 = 2u * (cc & 3u);
+      st_shared_v4(base + ((q0 ^ swz) << 4), e4m3x2_times_f32(w[c][0], scale), e4m3x2_times_f32(w[c][0] >> 16, scale),
+                   e4m3x2_times_f32(w[c][1], scale), e4m3x2_times_f32(w[c][1] >> 16, scale));
+      st_shared_v4(base + (((q0 + 1u) ^ swz) << 4), e4m3x2_times_f32(w[c][2], scale),
+                   e4m3x2_times_f32(w[c][2] >> 16, scale), e4m3x2_times_f32(w[c][3], scale),
+                   e4m3x2_times_f32(w[c][3] >> 16, scale));
+    }
+  }
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                           const __grid_constant__ CUtensorMap tm_scale, const __grid_constant__ CUtensorMap tm_rope,
                            const DecodeParams p) {
+  using C = PairCfg<FP8>;
+  constexpr int kNumSlots = C::kNumSlots;
+  constexpr uint32_t kIdescQK = C::kIdescQK;
+  constexpr uint32_t kIdescPV = C::kIdescPV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + kOffQ;
   const uint32_t sP = sbase + kOffP;
   const uint32_t sSlots = sbase + kOffSlots;
-  const uint32_t sRope = sbase + kOffRope;
-  uint8_t* misc = smem + kOffMisc;
+  const uint32_t sRope = sbase + C::kOffRope;
+  const uint32_t sRaw = sbase + C::kOffRaw;
+  uint8_t* misc = smem + C::kOffMisc;
   const uint32_t sMisc = smem_u32(misc);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + kMiscHolder);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + kMiscAbort);
@@ -270,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarZFull + i), 8);
       mbar_init(bar(kBarZLocal + i), 1);
     }
-    mbar_init(bar(kBarRopeFull), 2);
+    mbar_init(bar(kBarRopeFull), FP8 ? 1 : 2);
     mbar_init(bar(kBarRopeEmpty), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
@@ -280,12 +387,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarPFull), 8);
     mbar_init(bar(kBarPRecv), 1);
     mbar_init(bar(kBarPEmpty), 1);
-    mbar_init(bar(kBarQFull), 2);
+    mbar_init(bar(kBarQFull), FP8 ? 1 : 2);
     mbar_init(bar(kBarQEmpty), 1);
     mbar_init(bar(kBarOFull), 1);
     mbar_init(bar(kBarOEmpty), 16);
     mbar_init(bar(kBarDrain), 1);
     mbar_init(bar(kBarLFull), 1);
+    for (int i = 0; i < kNumRaw; ++i) {
+      mbar_init(bar(kBarRawFull + i), 1);
+      mbar_init(bar(kBarRawEmpty + i), 1);
+    }
+    mbar_init(bar(kBarQReady), 2);
+    mbar_init(bar(kBarRopeReady), 2);
     *abort_flag = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerFills) = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerQ) = 0;
@@ -295,6 +408,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpProducer && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_kv);
+    if (FP8) {
+      tma_prefetch_desc(&tm_scale);
+      tma_prefetch_desc(&tm_rope);
+    }
   }
   if (warp == kWarpMma) {
     tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
@@ -357,16 +474,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++fills;
         return true;
       };
+      // FP8: one stage's raw data = the 128 code bytes at byte cx of two pages (py, valid pv) and
+      // their scales, into this CTA's raw ring ([page][64 tokens][128 B] codes, then
+      // [page][64 tokens][16 B] scales), counted on this CTA's own barrier.
+      int last_raw[kNumRaw];
+      for (int i = 0; i < kNumRaw; ++i) last_raw[i] = -1;
+      auto fill_raw = [&](int cx, const int* py, const bool* pv, uint64_t pol) -> bool {
+        const int r = static_cast<int>(fills % kNumRaw);
+        const uint32_t use = fills / kNumRaw;
+        if (!pwait(bar(kBarRawEmpty + r), (use & 1u) ^ 1u, wc)) return false;
+        const uint32_t full = bar(kBarRawFull + r);
+        const uint32_t np = (pv[0] ? 1u : 0u) + (pv[1] ? 1u : 0u);
+        mbar_arrive_expect_tx(full, np * (kRawCodeBytes / 2 + kRawScaleBytes / 2));
+        const uint32_t dst = sRaw + static_cast<uint32_t>(r) * kRawBytes;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          if (!pv[q]) continue;
+          tma_load_2d(dst + q * (kRawCodeBytes / 2), &tm_kv, cx, py[q], full, pol);
+          tma_load_2d(dst + kRawCodeBytes + q * (kRawScaleBytes / 2), &tm_scale, kDv, py[q], full, pol);
+        }
+        last_raw[r] = static_cast<int>(use);
+        ++fills;
+        return true;
+      };
       while (ok && walk.next(p, b, c0, c1, split)) {
         const int L = p.cache_seqlens[b];
         const int npages = (L + kPage - 1) / kPage;
         const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
         if (!pwait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc)) break;
-        const uint32_t qfull = lead(bar(kBarQFull));
-        mbar_arrive_expect_tx_relaxed(qfull, static_cast<uint32_t>(kQBytes));
-        for (int a = 0; a < 9; ++a)
-          tma_load_3d_pair(sQ + a * kBoxBytes, &tm_q, 64 * a, rg * kRows + static_cast<int>(rank) * kHalfRows, b,
-                           qfull);
+        if (FP8) {
+          // this CTA's copy; its dequant warps convert Q to f16 before the leader's MMA uses it
+          mbar_arrive_expect_tx(bar(kBarQFull), static_cast<uint32_t>(kQBytes));
+          for (int a = 0; a < 9; ++a)
+            tma_load_3d(sQ + a * kBoxBytes, &tm_q, 64 * a, rg * kRows + static_cast<int>(rank) * kHalfRows, b,
+                        bar(kBarQFull));
+        } else {
+          const uint32_t qfull = lead(bar(kBarQFull));
+          mbar_arrive_expect_tx_relaxed(qfull, static_cast<uint32_t>(kQBytes));
+          for (int a = 0; a < 9; ++a)
+            tma_load_3d_pair(sQ + a * kBoxBytes, &tm_q, 64 * a, rg * kRows + static_cast<int>(rank) * kHalfRows, b,
+                             qfull);
+        }
         ++q_fills;
         const int n = (c1 - c0 + 1) / 2;
         for (int e = 0; ok && e < 2 * n; ++e) {
@@ -384,18 +532,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               // the RoPE dims first: QK(t) starts with them
               const uint32_t use = static_cast<uint32_t>(rope_fills);
               if (!pwait(bar(kBarRopeEmpty), (use & 1u) ^ 1u, wc)) { ok = false; break; }
-              const uint32_t rfull = lead(bar(kBarRopeFull));
-              mbar_arrive_expect_tx_relaxed(rfull, static_cast<uint32_t>(((va ? 1 : 0) + (vb ? 1 : 0)) * kBoxBytes));
-              if (va) tma_load_2d_pair(sRope, &tm_kv, kDv, ya, rfull, pol_rope);
-              if (vb) tma_load_2d_pair(sRope + kBoxBytes, &tm_kv, kDv, yb, rfull, pol_rope);
+              const uint32_t rbytes = static_cast<uint32_t>(((va ? 1 : 0) + (vb ? 1 : 0)) * kBoxBytes);
+              if (FP8) {
+                // the bf16 RoPE bytes of the 656-byte tokens, into this CTA (converted to f16 there)
+                mbar_arrive_expect_tx(bar(kBarRopeFull), rbytes);
+                if (va) tma_load_2d(sRope, &tm_rope, kDv + 16, ya, bar(kBarRopeFull), pol_rope);
+                if (vb) tma_load_2d(sRope + kBoxBytes, &tm_rope, kDv + 16, yb, bar(kBarRopeFull), pol_rope);
+              } else {
+                const uint32_t rfull = lead(bar(kBarRopeFull));
+                mbar_arrive_expect_tx_relaxed(rfull, rbytes);
+                if (va) tma_load_2d_pair(sRope, &tm_kv, kDv, ya, rfull, pol_rope);
+                if (vb) tma_load_2d_pair(sRope + kBoxBytes, &tm_kv, kDv, yb, rfull, pol_rope);
+              }
               ++rope_fills;
             }
             for (int j = 0; ok && j < kKFills; ++j) {
               // half h = dims 128j + 64h .. +63 of both pages (page a at +0, page b at +8 KB)
-              const int x[4] = {128 * j, 128 * j, 128 * j + 64, 128 * j + 64};
-              const int yy[4] = {ya, yb, ya, yb};
-              const bool vv[4] = {va, vb, va, vb};
-              ok = fill(x, yy, vv, pol_keep, false);
+              if (FP8) {
+                const int py[2] = {ya, yb};
+                const bool pv[2] = {va, vb};
+                ok = fill_raw(128 * j, py, pv, pol_keep);
+              } else {
+                const int x[4] = {128 * j, 128 * j, 128 * j + 64, 128 * j + 64};
+                const int yy[4] = {ya, yb, ya, yb};
+                const bool vv[4] = {va, vb, va, vb};
+                ok = fill(x, yy, vv, pol_keep, false);
+              }
             }
           } else {
             // V(t): this CTA's 256 output dims of the step's two token blocks; stage (m, blk) holds
@@ -412,10 +574,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int m = 0; ok && m < 2; ++m) {
               const int d = 256 * m + 128 * static_cast<int>(rank);
               for (int blk = 0; ok && blk < 2; ++blk) {
-                const int x[4] = {d, d + 64, d, d + 64};
-                const int yy[4] = {y[2 * blk], y[2 * blk], y[2 * blk + 1], y[2 * blk + 1]};
-                const bool vv[4] = {v[2 * blk], v[2 * blk], v[2 * blk + 1], v[2 * blk + 1]};
-                ok = fill(x, yy, vv, pol_v, tail);
+                if (FP8) {
+                  const int py[2] = {y[2 * blk], y[2 * blk + 1]};
+                  const bool pv[2] = {v[2 * blk], v[2 * blk + 1]};
+                  ok = fill_raw(d, py, pv, pol_v);
+                } else {
+                  const int x[4] = {d, d + 64, d, d + 64};
+                  const int yy[4] = {y[2 * blk], y[2 * blk], y[2 * blk + 1], y[2 * blk + 1]};
+                  const bool vv[4] = {v[2 * blk], v[2 * blk], v[2 * blk + 1], v[2 * blk + 1]};
+                  ok = fill(x, yy, vv, pol_v, tail);
+                }
               }
             }
           }
@@ -427,12 +595,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_use[s] >= 0) drain_wait(bar(kBarSlotEmpty + s), static_cast<uint32_t>(last_use[s]) & 1u);
         if (q_fills > 0) drain_wait(bar(kBarQEmpty), static_cast<uint32_t>(q_fills - 1) & 1u);
         if (rope_fills > 0) drain_wait(bar(kBarRopeEmpty), static_cast<uint32_t>(rope_fills - 1) & 1u);
+      } else if (FP8) {
+        // every copy of an FP8 CTA counts on its own barriers: let the last ones land
+        for (int r = 0; r < kNumRaw; ++r)
+          if (last_raw[r] >= 0) drain_wait(bar(kBarRawFull + r), static_cast<uint32_t>(last_raw[r]) & 1u);
+        if (q_fills > 0) drain_wait(bar(kBarQFull), static_cast<uint32_t>(q_fills - 1) & 1u);
+        if (rope_fills > 0) drain_wait(bar(kBarRopeFull), static_cast<uint32_t>(rope_fills - 1) & 1u);
       } else {
         // copies of tail V slots count on this CTA's own barriers: let them land
         for (int s = 0; s < kNumSlots; ++s)
           if ((zl_uses >> s) & 1u) drain_wait(bar(kBarZLocal + s), ((zl_par >> s) & 1u) ^ 1u);
       }
-      if (!leader) {
+      if (!FP8 && !leader) {
         st_cluster_u32(lead(sMisc + kMiscPeerFills), fills);
         st_cluster_u32(lead(sMisc + kMiscPeerQ), static_cast<uint32_t>(q_fills));
         st_cluster_u32(lead(sMisc + kMiscPeerRope), static_cast<uint32_t>(rope_fills));
@@ -459,7 +633,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok && walk.next(p, b, c0, c1, split)) {
         const int L = p.cache_seqlens[b];
         const int n = (c1 - c0 + 1) / 2;
-        if (!pwait(bar(kBarQFull), chunk & 1, wc)) break;
+        // FP8: both CTAs' dequant warps have converted their Q halves to f16
+        if (!pwait(bar(FP8 ? kBarQReady : kBarQFull), chunk & 1, wc)) break;
         for (int e = 0; ok && e < 2 * n; ++e) {
           bool is_v;
           int t;
@@ -470,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!pwait(bar(kBarSEmpty + sb), ((u >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
             const uint32_t d = tmem + kColS + 128u * sb;
             // RoPE dims first (they have their own slot), then the four 128-dim K stages
-            if (!pwait(bar(kBarRopeFull), rope_used & 1u, wc)) { ok = false; break; }
+            if (!pwait(bar(FP8 ? kBarRopeReady : kBarRopeFull), rope_used & 1u, wc)) { ok = false; break; }
             ++rope_used;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -501,7 +676,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // tcgen05 fence in the issue stream drains the MMA pipe, so none sits before
             // operands that only TMA or shared-memory stores produced
             tc_fence_after();
-            const bool tail = is_tail(c0, c1, t, L);
+            // FP8 stages hold zeros for tokens outside the request (written by the dequant warps)
+            const bool tail = !FP8 && is_tail(c0, c1, t, L);
             for (int m = 0; ok && m < 2; ++m) {
               for (int blk = 0; blk < 2; ++blk) {
                 uint32_t s;
@@ -534,6 +710,106 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every pair MMA is complete before tensor memory is released
       umma_commit_pair(bar(kBarDrain));
       drain_wait(bar(kBarDrain), 0);
+    }
+  } else if (FP8 && warp >= kWarpDequant) {
+    // =========================== FP8 dequant (warps 10-13) ===========================
+    // Thread dt owns token row dt % 64 of page dt / 64 of each stage.  Order: per chunk the Q
+    // tile, then the stages in the fill order, each K step preceded by its RoPE slot.
+    if (warp < kWarpDequant + kDequantThreads / 32) {
+    const int dt = threadIdx.x - kWarpDequant * 32;  // 0..127
+    uint32_t g = 0;   // stages written
+    uint32_t gr = 0;  // raw fills consumed
+    uint32_t qc = 0, rc = 0;
+    int last_use[kMaxSlots];
+    for (int i = 0; i < kMaxSlots; ++i) last_use[i] = -1;
+    bool ok = true;
+    // bf16 -> f16 in place over `bytes` of shared memory at `base`
+    auto to_f16 = [&](uint32_t base, int bytes) {
+      for (int c = dt; c < bytes / 16; c += kDequantThreads) {
+        uint32_t w0, w1, w2, w3;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                     : "r"(base + 16u * c));
+        st_shared_v4(base + 16u * c, bf16x2_to_f16x2(w0), bf16x2_to_f16x2(w1), bf16x2_to_f16x2(w2),
+                     bf16x2_to_f16x2(w3));
+      }
+    };
+    // publish this CTA's f16 data to the leader's MMA: count-2 barrier `b` of the leader
+    auto publish = [&](int b) -> bool {
+      fence_proxy_async_smem();
+      if (named_bar_any(3, kDequantThreads, !ok)) return false;
+      if (dt == 0) mbar_arrive_remote(lead(bar(b)));
+      return true;
+    };
+    // one stage: kind V (else K), token block tb of the step, scale group grp; page p of the
+    // stage lands at +p * pstride, dim half h at +h * hstride
+    auto stage = [&](int tb, int c1, int L, int grp, uint32_t pstride, uint32_t hstride) -> bool {
+      const uint32_t s = g % kNumSlots;
+      const uint32_t use = g / kNumSlots;
+      const uint32_t r = gr % kNumRaw;
+      ok &= warp_pwait(bar(kBarRawFull + r), (gr / kNumRaw) & 1u, wc, lane);
+      ok &= warp_pwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc, lane);
+      if (ok) {
+        const uint32_t raw = sRaw + r * kRawBytes;
+        const uint32_t pg = static_cast<uint32_t>(dt) >> 6, i = static_cast<uint32_t>(dt) & 63u;
+        const uint32_t dst = sSlots + s * kSlotBytes + pg * pstride + i * 128u;
+        const int tok = tb * kBlockTokens + dt;  // page pg, row i
+        if (tb < c1 && tok < L) {
+          float scale;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(scale)
+                       : "r"(raw + kRawCodeBytes + pg * (kRawScaleBytes / 2) + i * 16u + 4u * grp));
+          dequant_row(raw + pg * (kRawCodeBytes / 2) + i * 128u, dst, hstride, i, scale);
+        } else {
+          // tokens outside the request or the chunk: zeros (masked in S^T, 0 rows of V)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) st_shared_v4(dst + h * hstride + 16u * q, 0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      if (named_bar_any(3, kDequantThreads, !ok)) return false;
+      if (dt == 0) {
+        mbar_arrive(bar(kBarRawEmpty + r));
+        mbar_arrive_remote(lead(bar(kBarSlotFull + s)));
+      }
+      last_use[s] = static_cast<int>(use);
+      ++g;
+      ++gr;
+      return true;
+    };
+    ChunkWalk walk(p, part);
+    int b, c0, c1, split;
+    while (ok && walk.next(p, b, c0, c1, split)) {
+      const int L = p.cache_seqlens[b];
+      const int n = (c1 - c0 + 1) / 2;
+      ok &= warp_pwait(bar(kBarQFull), qc & 1u, wc, lane);
+      if (ok) to_f16(sQ, kQBytes);
+      ++qc;
+      if (!publish(kBarQReady)) break;
+      for (int e = 0; ok && e < 2 * n; ++e) {
+        bool is_v;
+        int t;
+        order_at(e, n, is_v, t);
+        if (!is_v) {
+          ok &= warp_pwait(bar(kBarRopeFull), rc & 1u, wc, lane);
+          if (ok) to_f16(sRope, kRopeBytes);
+          ++rc;
+          if (!publish(kBarRopeReady)) { ok = false; break; }
+          // K(t) stage j: dims 128j.. of this CTA's block; [dim half][page][64 tokens][64 dims]
+          for (int j = 0; ok && j < kKFills; ++j)
+            ok = stage(c0 + 2 * t + static_cast<int>(rank), c1, L, j, kBoxBytes, kHalfBytes);
+        } else {
+          // V(t) stage (m, blk): dims 256m + 128 rank.. of block c0 + 2t + blk; [page][dim half][..]
+          for (int k = 0; ok && k < kVFills; ++k)
+            ok = stage(c0 + 2 * t + (k & 1), c1, L, 2 * (k >> 1) + static_cast<int>(rank), kHalfBytes, kBoxBytes);
+        }
+      }
+    }
+    if (!*abort_flag && lane == 0)
+      // the last pair commits on this CTA's stage barriers have landed before it may exit
+      for (int s = 0; s < kNumSlots; ++s)
+        if (last_use[s] >= 0) drain_wait(bar(kBarSlotEmpty + s), static_cast<uint32_t>(last_use[s]) & 1u);
+    __syncwarp();
     }
   } else {
     // ============================ softmax + epilogue ==============================
@@ -658,8 +934,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q8 = 0; q8 < 8; ++q8) {
           const uint32_t off = T * 128u + ((static_cast<uint32_t>(q8) ^ (T & 7u)) << 4);
           const float* xs = x + 8 * q8;
-          const uint32_t w0 = pack_bf16x2(xs[0], xs[1]), w1 = pack_bf16x2(xs[2], xs[3]);
-          const uint32_t w2 = pack_bf16x2(xs[4], xs[5]), w3 = pack_bf16x2(xs[6], xs[7]);
+          uint32_t w0, w1, w2, w3;
+          if (FP8) {
+            w0 = pack_f16x2(xs[0], xs[1]), w1 = pack_f16x2(xs[2], xs[3]);
+            w2 = pack_f16x2(xs[4], xs[5]), w3 = pack_f16x2(xs[6], xs[7]);
+          } else {
+            w0 = pack_bf16x2(xs[0], xs[1]), w1 = pack_bf16x2(xs[2], xs[3]);
+            w2 = pack_bf16x2(xs[4], xs[5]), w3 = pack_bf16x2(xs[6], xs[7]);
+          }
           if (local) st_shared_v4(sP + off, w0, w1, w2, w3);
           else st_async_v4(other(sP + off), w0, w1, w2, w3, other(bar(kBarPRecv)));
         }
@@ -677,7 +959,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ok &= __shfl_sync(0xffffffffu, okp, 0) != 0;
         }
-        if (tid < kRows && is_tail(c0, c1, t, L)) {
+        if (!FP8 && tid < kRows && is_tail(c0, c1, t, L)) {
           // Zero, in this CTA's V slots of the step, the rows of tokens outside the request or the
           // chunk (stale ring contents or the cache's unused page tail: 0 * NaN would poison O^T).
           // These slots count their bytes on this CTA's own barrier; both CTAs then arrive on the
@@ -774,7 +1056,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();
-  if (leader && warp == kWarpProducer && lane == 0 && *abort_flag) {
+  if (!FP8 && leader && warp == kWarpProducer && lane == 0 && *abort_flag) {
     // After an abort, complete on behalf of the CTA that stopped first the fills the other one
     // issued, and wait for every copy still in flight into either CTA (the follower's copies
     // count their bytes here).  The two producers are at most one ring apart.
@@ -815,15 +1097,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
-                            cudaStream_t stream) {
-  auto kern = mla_decode_pair_kernel;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+template <bool FP8>
+int launch_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_scale,
+                const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
+  using C = PairCfg<FP8>;
+  auto kern = mla_decode_pair_kernel<FP8>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return static_cast<int>(e);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * p.num_sm_parts, p.row_groups, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -832,8 +1116,18 @@ int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, c
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_kv, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_kv, tm_scale, tm_rope, p);
   return static_cast<int>(e);
+}
+
+int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
+                            cudaStream_t stream) {
+  return launch_pair<false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+}
+
+int launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
+                           const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
+  return launch_pair<true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
 }
 
 }  // namespace mla

@@ -57,9 +57,9 @@ struct CombineParams {
 inline int row_groups_for(int rows) { return rows <= kRowsPerCta ? 1 : (rows + kRowsPerCta - 1) / kRowsPerCta; }
 
 // Requests with more than 64 query rows run on CTA pairs of 128 rows each (mla_decode_pair.cu,
-// bf16 cache); a scheduler part then needs 2 SMs per 128-row group.
+// bf16 or FP8 cache); a scheduler part then needs 2 SMs per 128-row group.
 constexpr int kPairRows = 128;
-inline bool use_pair_kernel(int rows, bool fp8) { return rows > kRowsPerCta && !fp8; }
+inline bool use_pair_kernel(int rows, bool /*fp8*/) { return rows > kRowsPerCta; }
 inline int sms_per_part(int rows) { return rows <= kRowsPerCta ? 1 : 2 * ((rows + kPairRows - 1) / kPairRows); }
 
 // launchers (return cudaError_t as int)
@@ -71,6 +71,8 @@ int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, cons
                       const CUtensorMap& tm_rope, const DecodeParams& p, int rows_per_cta, cudaStream_t stream);
 int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
                             cudaStream_t stream);
+int launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
+                           const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream);
 int launch_combine(const CombineParams& p, cudaStream_t stream);
 
 }  // namespace mla
