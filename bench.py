@@ -331,7 +331,9 @@ def main():
     line = {
         "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "data": "synthetic",
+        # the arithmetic type of the MMAs: FP8 caches above 64 query rows run on f16 operands
+        "dtype": "f16" if case.kv_format == "fp8" and case.s_q * case.h_q > 64 else "bf16",
         "config": {"workload": args.workload, "batch": case.batch, "s_q": case.s_q, "h_q": case.h_q,
                    "h_kv": 1, "d_qk": 576, "d_v": 512, "page": 64, "seqlens": w.seqlens, "causal": case.causal,
                    "kv": case.kv_format, "kv_bytes": units["kv_bytes"], "l2": "inputs larger than L2 (no flush)",

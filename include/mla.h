@@ -113,7 +113,10 @@ MLA_API size_t mla_workspace_size(int batch, int num_sm_parts, int rows_per_kv_h
  *   tile_md, num_splits   from mla_get_metadata with the same cache_seqlens and num_sm_parts
  *   softmax_scale  multiplies q.k (e.g. 576^-0.5)
  *   causal         0 / 1
- *   kv_dtype       MLA_KV_BF16 or MLA_KV_FP8
+ *   kv_dtype       MLA_KV_BF16 or MLA_KV_FP8.  With MLA_KV_FP8 and more than 64 query rows per
+ *                  request the products run on f16 tensor cores: q, the RoPE dims and every
+ *                  code * scale must stay within the f16 range (|x| < 65504; scales up to 146);
+ *                  e4m3 NaN codes are not expected (a quantised cache holds none)
  *   out            device bf16 [batch, s_q, h_q, 512] (written)
  *   lse            device fp32 [batch, h_q, s_q] (written)
  *   workspace      device scratch of >= mla_workspace_size(batch, num_sm_parts, s_q*h_q, h_kv) bytes,
