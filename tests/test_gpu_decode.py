@@ -210,6 +210,26 @@ def test_parity_fp8_small(name, batch, s_q, h_q, seqlens, causal, parts):
     compare(case, out, lse, O_ref, L_ref)
 
 
+@pytest.mark.parametrize("h_q", [16, 128])
+def test_fp8_small_scales(h_q):
+    """Scales below 2^-14 (the f16 normal range) take the fp32 product in the dequant of the
+    CTA-pair path.  The case is the unit case with every scale and RoPE value times 2^-10 and
+    the softmax scale times 2^10: the same softmax, O times 2^-10 (compared at unit scale)."""
+    case = mi.make_case(2, 1, h_q, [300, 1000], kv_format="fp8", seed=57, spare_blocks=2)
+    kv = case.kv.reshape(-1, mi.FP8_TOKEN_BYTES)
+    scales = kv[:, 512:528].copy().view(np.float32) * np.float32(2.0 ** -10)
+    kv[:, 512:528] = scales.view(np.uint8)
+    rope = kv[:, 528:656].copy().view(np.uint16).astype(np.uint32) << 16
+    rope = (rope.view(np.float32) * np.float32(2.0 ** -10)).view(np.uint32) >> 16
+    kv[:, 528:656] = rope.astype(np.uint16).view(np.uint8)
+    assert float(np.nanmax(scales)) < 2.0 ** -14
+    case.softmax_scale = case.softmax_scale * 2.0 ** 10
+    O_ref, L_ref = oracle.mla_decode_reference(case)
+    out, lse, status, _ = run_gpu(case)
+    assert status == 0
+    compare(case, out.astype(np.float64) * 2.0 ** 10, lse, O_ref * 2.0 ** 10, L_ref)
+
+
 def test_fp8_nan_in_unreadable_slots_does_not_leak():
     clean = mi.make_case(2, 1, 128, [70, 129], kv_format="fp8", seed=31, poison=False, spare_blocks=3)
     dirty = mi.make_case(2, 1, 128, [70, 129], kv_format="fp8", seed=31, poison=True, spare_blocks=3)
