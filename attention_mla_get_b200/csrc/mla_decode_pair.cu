@@ -112,7 +112,7 @@ constexpr int kMaxSlots = 3;
 
 // misc area: barriers, then scalars, then per-row scratch
 enum : int {
-  // [stages] leader: both producers (FP8: both dequant groups), count 2 + bytes
+  // [stages] leader: both producers, count 2 + bytes (FP8: every dequant warp of both CTAs)
   kBarSlotFull = 0,
   kBarSlotEmpty = kBarSlotFull + kMaxSlots,   // [stages] both: pair commit
   kBarZFull = kBarSlotEmpty + kMaxSlots,      // [stages] leader: both CTAs zeroed a tail V slot
@@ -133,9 +133,9 @@ enum : int {
   kBarLFull = kBarMaxFull + 2,                // both: 512 bytes of the peer's row sums
   kBarPRecv = kBarLFull + 1,                  // both: 16 KB of P^T rows from the peer
   kBarRawFull = kBarPRecv + 1,                // [2] FP8, both: this CTA's raw fill, count 1 + bytes
-  kBarRawEmpty = kBarRawFull + kNumRaw,       // [2] FP8, both: this CTA's dequant group
-  kBarQReady = kBarRawEmpty + kNumRaw,        // FP8, leader: Q in f16 in both CTAs, count 2
-  kBarRopeReady = kBarQReady + 1,             // FP8, leader: RoPE slot in f16 in both CTAs, count 2
+  kBarRawEmpty = kBarRawFull + kNumRaw,       // [2] FP8, both: this CTA's dequant warps
+  kBarQReady = kBarRawEmpty + kNumRaw,        // FP8, leader: Q in f16 (every dequant warp, both CTAs)
+  kBarRopeReady = kBarQReady + 1,             // FP8, leader: RoPE slot in f16 (as kBarQReady)
   kNumBars = kBarRopeReady + 1,
 };
 constexpr int kMiscHolder = 512;   // TMEM base address
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumSlots; ++i) {
-      mbar_init(bar(kBarSlotFull + i), 2);
+      mbar_init(bar(kBarSlotFull + i), FP8 ? 2 * kDequantThreads / 32 : 2);
       mbar_init(bar(kBarSlotEmpty + i), 1);
       mbar_init(bar(kBarZFull + i), 8);
       mbar_init(bar(kBarZLocal + i), 1);
@@ -395,10 +395,10 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
     mbar_init(bar(kBarLFull), 1);
     for (int i = 0; i < kNumRaw; ++i) {
       mbar_init(bar(kBarRawFull + i), 1);
-      mbar_init(bar(kBarRawEmpty + i), 1);
+      mbar_init(bar(kBarRawEmpty + i), kDequantThreads / 32);
     }
-    mbar_init(bar(kBarQReady), 2);
-    mbar_init(bar(kBarRopeReady), 2);
+    mbar_init(bar(kBarQReady), 2 * kDequantThreads / 32);
+    mbar_init(bar(kBarRopeReady), 2 * kDequantThreads / 32);
     *abort_flag = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerFills) = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerQ) = 0;
@@ -733,11 +733,12 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
                      bf16x2_to_f16x2(w3));
       }
     };
-    // publish this CTA's f16 data to the leader's MMA: count-2 barrier `b` of the leader
+    // publish this warp's f16 data to the leader's MMA (each dequant warp of both CTAs arrives)
     auto publish = [&](int b) -> bool {
       fence_proxy_async_smem();
-      if (named_bar_any(3, kDequantThreads, !ok)) return false;
-      if (dt == 0) mbar_arrive_remote(lead(bar(b)));
+      __syncwarp();
+      if (!ok) return false;
+      if (lane == 0) mbar_arrive_remote(lead(bar(b)));
       return true;
     };
     // one stage: kind V (else K), token block tb of the step, scale group grp; page p of the
@@ -767,8 +768,9 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      if (named_bar_any(3, kDequantThreads, !ok)) return false;
-      if (dt == 0) {
+      __syncwarp();
+      if (!ok) return false;
+      if (lane == 0) {
         mbar_arrive(bar(kBarRawEmpty + r));
         mbar_arrive_remote(lead(bar(kBarSlotFull + s)));
       }
