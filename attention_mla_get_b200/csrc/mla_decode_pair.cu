@@ -615,7 +615,6 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
   } else if (warp == kWarpMma) {
     // ================================ MMA issuer (leader) =========================
     if (leader && lane == 0) {
-      uint32_t g = 0;   // slot fills consumed
       uint32_t u = 0;   // QK steps issued
       uint32_t up = 0;  // PV steps issued
       uint32_t rope_used = 0;
@@ -624,12 +623,19 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
       bool ok = true;
       ChunkWalk walk(p, part);
       int b, c0, c1, split;
+      uint32_t gs = 0, gph = 0;  // slot of the next fill to consume, and its phase parity
       auto next_slot = [&](uint32_t& s) -> bool {
-        s = g % kNumSlots;
-        if (!pwait(bar(kBarSlotFull + s), (g / kNumSlots) & 1u, wc)) return false;
-        ++g;
+        s = gs;
+        if (!pwait(bar(kBarSlotFull + s), gph, wc)) return false;
+        if (++gs == static_cast<uint32_t>(kNumSlots)) {
+          gs = 0;
+          gph ^= 1u;
+        }
         return true;
       };
+      // shared-memory descriptors of stage 0; stage s adds s * kSlotBytes >> 4
+      const uint64_t kdesc0 = smem_desc(sSlots, 16, 1024, kSwizzle128);
+      const uint64_t vdesc0 = smem_desc(sSlots, kBoxBytes, 1024, kSwizzle128);
       while (ok && walk.next(p, b, c0, c1, split)) {
         const int L = p.cache_seqlens[b];
         const int n = (c1 - c0 + 1) / 2;
@@ -657,7 +663,7 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
               uint32_t s;
               if (!next_slot(s)) { ok = false; break; }
               // descriptors advance by (byte offset >> 4) in their start-address field
-              const uint64_t a0 = smem_desc(sSlots + s * kSlotBytes, 16, 1024, kSwizzle128);
+              const uint64_t a0 = kdesc0 + static_cast<uint64_t>(s * (kSlotBytes >> 4));
               const uint64_t b0 = smem_desc(sQ + 2 * j * kBoxBytes, 16, 1024, kSwizzle128);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
@@ -687,7 +693,7 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
                   zpar ^= 1u << s;
                 }
                 // half h = page 2 blk + h of the step (64 tokens x 128 dims, 64-dim boxes 8 KB apart)
-                const uint64_t a0 = smem_desc(sSlots + s * kSlotBytes, kBoxBytes, 1024, kSwizzle128);
+                const uint64_t a0 = vdesc0 + static_cast<uint64_t>(s * (kSlotBytes >> 4));
                 const uint64_t b0 = smem_desc(sP + 128 * blk * 128, kBoxBytes, 1024, kSwizzle128);
 #pragma unroll
                 for (int kt = 0; kt < 8; ++kt)
