@@ -45,7 +45,7 @@ E4M3_NAN = np.uint8(0x7F)
 _CHUNK_ELEMS = 1 << 22   # elements per random chunk (fixed: keeps results thread-count independent)
 
 # random stream ids
-_S_SEQLENS, _S_PERM, _S_Q, _S_KV = 0, 1, 2, 3
+_S_SEQLENS, _S_PERM, _S_Q, _S_KV, _S_IDX = 0, 1, 2, 3, 4
 
 
 @dataclass
@@ -63,6 +63,11 @@ class DecodeCase:
     h_kv: int = 1
     name: str = ""
     meta: dict = field(default_factory=dict)
+    indices: Optional[np.ndarray] = None   # token-sparse decode: int32 [b, s_q, topk], else None
+
+    @property
+    def topk(self) -> int:
+        return 0 if self.indices is None else int(self.indices.shape[-1])
 
     @property
     def batch(self) -> int:
@@ -96,6 +101,7 @@ class Workload:
     kv_format: str
     seed: int
     description: str
+    topk: int = 0                 # > 0: token-sparse decode over topk cache positions per query
 
 
 WORKLOADS = {
@@ -114,6 +120,10 @@ WORKLOADS = {
     "fp8_b128_h128_L16384": Workload(
         "fp8_b128_h128_L16384", 128, 1, 128, "fixed:16384", False, "fp8", 5,
         "FP8 KV decode: batch 128, s_q 1, h_q 128, every cache_seqlen 16384, 656-byte tokens"),
+    "sparse_b128_h128_L8192_topk2048": Workload(
+        "sparse_b128_h128_L8192_topk2048", 128, 1, 128, "fixed:8192", False, "bf16", 6,
+        "token-sparse decode: batch 128, s_q 1, h_q 128, every cache_seqlen 8192, 2048 distinct "
+        "cache positions per query in random order", topk=2048),
 }
 
 
@@ -284,6 +294,34 @@ def make_case(batch: int, s_q: int, h_q: int, cache_seqlens: Sequence[int] | np.
     return case
 
 
+def make_sparse_indices(cache_seqlens, s_q: int, topk: int, seed: int, *, invalid_frac: float = 0.0,
+                        duplicate_frac: float = 0.0) -> np.ndarray:
+    """Seeded index lists int32 [b, s_q, topk] for token-sparse decode.
+
+    Each (request b, query i) lists min(topk, L_b) distinct cache positions of [0, L_b) in
+    random order, then -1 for the remaining slots.  Optionally a fraction of the entries is
+    replaced by an empty-slot value (-1, or a position >= L_b) and a fraction by a copy of
+    another entry of the same list (a position counted twice)."""
+    L = np.asarray(cache_seqlens, dtype=np.int64).reshape(-1)
+    B = L.shape[0]
+    g = _seq(seed, _S_IDX)
+    out = np.full((B, s_q, topk), -1, dtype=np.int32)
+    for b in range(B):
+        for i in range(s_q):
+            n = int(min(topk, max(L[b], 0)))
+            if n > 0:
+                out[b, i, :n] = g.permutation(int(L[b]))[:n]
+            if invalid_frac > 0:
+                m = g.random(topk) < invalid_frac
+                bad = np.where(g.random(topk) < 0.5, -1, L[b] + g.integers(0, 1000, size=topk))
+                out[b, i, m] = bad[m].astype(np.int32)
+            if duplicate_frac > 0 and topk > 1:
+                m = g.random(topk) < duplicate_frac
+                src = g.integers(0, topk, size=topk)
+                out[b, i, m] = out[b, i, src[m]]
+    return out
+
+
 def make_workload(name: str, *, batch: Optional[int] = None, poison: bool = True,
                   spare_blocks: int = 0) -> DecodeCase:
     """One of the named decode workloads at its full size (or with ``batch`` requests:
@@ -296,6 +334,8 @@ def make_workload(name: str, *, batch: Optional[int] = None, poison: bool = True
     case = make_case(b, w.s_q, w.h_q, seqlens, causal=w.causal, kv_format=w.kv_format, seed=w.seed,
                      spare_blocks=spare_blocks, poison=poison, name=name)
     case.meta["workload"] = w.description
+    if w.topk > 0:
+        case.indices = make_sparse_indices(case.cache_seqlens, w.s_q, w.topk, w.seed)
     return case
 
 
@@ -304,6 +344,15 @@ def workload_units(case: DecodeCase) -> dict:
     page-rounded), q/out/lse bytes and the FLOPs of the visible (row, key) pairs."""
     L = case.cache_seqlens.astype(np.int64)
     R = case.rows
+    if case.indices is not None:
+        # token-sparse: each query position reads and attends to its valid listed positions
+        valid = (case.indices >= 0) & (case.indices < L[:, None, None])
+        n_sel = int(valid.sum())
+        kv_bytes = n_sel * case.kv_bytes_per_token()
+        qob = case.batch * R * (D_QK * 2 + D_V * 2 + 4) + case.indices.size * 4
+        pairs = n_sel * case.h_q
+        return {"kv_bytes": kv_bytes, "kv_bytes_paged": kv_bytes, "bytes": kv_bytes + qob,
+                "qol_bytes": qob, "flops": 2 * (D_QK + D_V) * pairs, "pairs": pairs, "tokens": n_sel}
     kv_tok = int(L.sum())
     kv_bytes = kv_tok * case.kv_bytes_per_token()
     kv_bytes_paged = int(((L + PAGE - 1) // PAGE).sum()) * PAGE * case.kv_bytes_per_token()
@@ -325,4 +374,5 @@ __all__ = [
     "D_QK", "D_V", "D_ROPE", "PAGE", "FP8_TOKEN_BYTES", "FP8_GROUP", "E4M3_MAX",
     "DecodeCase", "Workload", "WORKLOADS", "make_case", "make_workload", "make_block_table",
     "draw_seqlens", "poison_unused", "f32_to_bf16_bits", "bf16_bits_to_f32", "workload_units",
+    "make_sparse_indices",
 ]

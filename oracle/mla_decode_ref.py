@@ -100,3 +100,40 @@ def mla_decode_reference(case, requests=None):
         O[b] = o.reshape(s_q, h_q, D_V)
         LSE[b] = l.reshape(s_q, h_q).T
     return O, LSE
+
+
+def mla_sparse_decode_reference(case, indices, requests=None):
+    """Token-sparse decode (the `indices` argument of flash_mla_with_kvcache and `topk` of
+    get_mla_metadata on the gitcode FlashMLA page, "解码阶段使用示例" / "稀疏解码场景"),
+    by definition, in fp64.
+
+    Reading (the page gives the call, not the shape): indices is int32 [b, s_q, topk];
+    query position i of request b attends to the tokens at the logical cache positions
+    indices[b, i, :] (addressed through block_table like every other key); an entry outside
+    [0, L_b) is an empty slot and contributes nothing; a position listed twice counts twice.
+    No causal mask applies (the index list already says what a query sees).
+
+      s_k  = softmax_scale * q[b, i, h] . K_b[indices[b, i, k]]       for valid k
+      LSE  = log sum_k exp(s_k),  O = sum_k exp(s_k - LSE) * K_b[indices[b, i, k]][:512]
+
+    Returns (O fp64 [b, s_q, h_q, 512], LSE fp64 [b, h_q, s_q]); a query with no valid
+    entry has O = 0 and LSE = -inf; requests not listed are NaN.
+    """
+    assert case.h_kv == 1, "the oracle follows the h_kv = 1 reading of the pages"
+    idx = np.asarray(indices)
+    B, s_q, h_q = case.batch, case.s_q, case.h_q
+    assert idx.ndim == 3 and idx.shape[:2] == (B, s_q), idx.shape
+    O = np.full((B, s_q, h_q, D_V), np.nan, dtype=np.float64)
+    LSE = np.full((B, h_q, s_q), np.nan, dtype=np.float64)
+    todo = range(B) if requests is None else requests
+    for b in todo:
+        L = int(case.cache_seqlens[b])
+        K = gather_request_keys(case, b)                             # [L, 576]
+        q = bf16_to_f64(case.q_bits[b])                              # [s_q, h_q, 576]
+        for i in range(s_q):
+            sel = [int(j) for j in idx[b, i] if 0 <= int(j) < L]
+            Ki = K[sel] if sel else np.zeros((0, D_QK), dtype=np.float64)
+            o, l = attend_rows(q[i], Ki, np.full(h_q, len(sel)), case.softmax_scale)
+            O[b, i] = o
+            LSE[b, :, i] = l
+    return O, LSE
