@@ -12,6 +12,10 @@ Calls (same names as the C-ABI):
     mla_workspace_size(batch, num_sm_parts, rows_per_kv_head, h_kv=1)
     mla_decode_kvcache(q, kvcache, block_table, cache_seqlens, d_v, tile_md, num_splits,
                        softmax_scale=None, causal=False, ...) -> (out bf16, lse fp32)
+    mla_get_metadata_sparse(batch, s_q, topk, h_q, h_kv=1, num_sm_parts=None)
+        -> (tile_md, num_splits int32 [batch * s_q + 1])        (token-sparse decode)
+    mla_decode_kvcache_sparse(q, kvcache, block_table, cache_seqlens, indices, d_v, tile_md,
+                              num_splits, softmax_scale=None) -> (out bf16, lse fp32)
     mla_read_status(workspace, reset=False)
 
 The FlashMLA-style spellings of the usage examples on the pages are provided too:
@@ -65,6 +69,11 @@ def _load() -> ctypes.CDLL:
     lib.mla_decode_kvcache.argtypes = [vp, vp, i64, vp, i32, vp, i32, i32, i32, i32, i32, vp, i32, vp,
                                        ctypes.c_float, i32, i32, vp, vp, vp, sz, vp]
     lib.mla_decode_kvcache.restype = i32
+    lib.mla_get_metadata_sparse.argtypes = [i32, i32, i32, i32, i32, vp, i32, vp, vp]
+    lib.mla_get_metadata_sparse.restype = i32
+    lib.mla_decode_kvcache_sparse.argtypes = [vp, vp, i64, vp, i32, vp, i32, i32, i32, i32, i32, vp, i32, vp, i32,
+                                              vp, ctypes.c_float, i32, vp, vp, vp, sz, vp]
+    lib.mla_decode_kvcache_sparse.restype = i32
     lib.mla_read_status.argtypes = [vp, i32, ctypes.POINTER(i32), vp]
     lib.mla_read_status.restype = i32
     lib.mla_strerror.argtypes = [i32]
@@ -77,7 +86,8 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 
 EXPORTED = ("mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-            "mla_decode_kvcache_noalloc", "mla_read_status", "mla_strerror", "mla_version")
+            "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
+            "mla_read_status", "mla_strerror", "mla_version")
 
 
 def mla_strerror(code: int) -> str:
@@ -179,6 +189,64 @@ def mla_decode_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torc
     return out, lse
 
 
+def mla_get_metadata_sparse(batch: int, s_q: int, topk: int, h_q: int, h_kv: int = 1,
+                            num_sm_parts: Optional[int] = None, device=None,
+                            stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Tile-scheduler metadata for token-sparse decode: batch * s_q query positions of topk
+    listed tokens each -> (tile_md int32 [num_sm_parts, 8], num_splits int32 [batch * s_q + 1])."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if num_sm_parts is None:
+        num_sm_parts = mla_num_sm_parts(h_q, h_kv, dev)
+    tile_md = torch.empty((num_sm_parts, 8), dtype=torch.int32, device=dev)
+    num_splits = torch.empty((batch * s_q + 1,), dtype=torch.int32, device=dev)
+    _check(_lib.mla_get_metadata_sparse(int(batch), int(s_q), int(topk), int(h_q), int(h_kv), _ptr(tile_md),
+                                        int(num_sm_parts), _ptr(num_splits), _stream(stream)),
+           "mla_get_metadata_sparse")
+    return tile_md, num_splits
+
+
+def mla_decode_kvcache_sparse(q: torch.Tensor, kvcache: torch.Tensor, block_table: torch.Tensor,
+                              cache_seqlens: torch.Tensor, indices: torch.Tensor, d_v: int, tile_md: torch.Tensor,
+                              num_splits: torch.Tensor, softmax_scale: Optional[float] = None,
+                              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None,
+                              stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Token-sparse MLA decode over indices int32 [b, s_q, topk] (bf16 cache):
+    returns (out bf16 [b, s_q, h_q, 512], lse fp32 [b, h_q, s_q])."""
+    if q.dtype != torch.bfloat16 or q.dim() != 4 or q.shape[-1] != D_QK:
+        raise ValueError("q must be bf16 [batch, s_q, h_q, 576]")
+    q = q.contiguous()
+    b, s_q, h_q, _ = q.shape
+    if kvcache.dtype != torch.bfloat16 or kvcache.shape[1] != PAGE or kvcache.shape[-1] != D_QK:
+        raise ValueError("kvcache must be bf16 [num_blocks, 64, (1,) 576] (token-sparse decode reads bf16 caches)")
+    if not kvcache.is_contiguous():
+        raise ValueError("kvcache must be contiguous")
+    h_kv = kvcache.shape[2] if kvcache.dim() == 4 else 1
+    if indices.dtype != torch.int32 or indices.dim() != 3 or tuple(indices.shape[:2]) != (b, s_q):
+        raise ValueError("indices must be int32 [batch, s_q, topk]")
+    indices = indices.contiguous()
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != b:
+        raise ValueError("block_table must be int32 [batch, max_blocks]")
+    block_table = block_table.contiguous()
+    topk = indices.shape[2]
+    if softmax_scale is None:
+        softmax_scale = D_QK ** -0.5
+    num_sm_parts = tile_md.shape[0]
+    if out is None:
+        out = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    need = mla_workspace_size(b * s_q, num_sm_parts, h_q, h_kv)
+    if workspace is None:
+        workspace = torch.zeros((max(need, 256),), dtype=torch.uint8, device=q.device)
+    _check(_lib.mla_decode_kvcache_sparse(
+        _ptr(q), _ptr(kvcache), kvcache.shape[0], _ptr(block_table), block_table.shape[1], _ptr(cache_seqlens),
+        b, s_q, h_q, h_kv, int(d_v), _ptr(indices), int(topk), _ptr(tile_md), num_sm_parts, _ptr(num_splits),
+        float(softmax_scale), KV_BF16, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)), "mla_decode_kvcache_sparse")
+    return out, lse
+
+
 def mla_read_status(workspace: torch.Tensor, reset: bool = False, stream=None) -> int:
     v = ctypes.c_int(0)
     _check(_lib.mla_read_status(_ptr(workspace), 1 if reset else 0, ctypes.byref(v), _stream(stream)),
@@ -200,6 +268,7 @@ def flash_mla_with_kvcache(q, k_cache, block_table, cache_seqlens, head_dim_v, t
 
 __all__ = [
     "mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache", "mla_read_status",
+    "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
     "mla_strerror", "mla_version", "get_mla_metadata", "flash_mla_with_kvcache", "MLAError", "LIB_PATH",
     "KV_BF16", "KV_FP8",
 ]

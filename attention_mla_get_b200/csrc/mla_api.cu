@@ -214,6 +214,100 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   return e == 0 ? MLA_OK : MLA_ERR_CUDA;
 }
 
+int mla_get_metadata_sparse(int batch, int s_q, int topk, int h_q, int h_kv, int32_t* tile_md, int num_sm_parts,
+                            int32_t* num_splits, void* stream) {
+  if (!tile_md || !num_splits) return MLA_ERR_NULL_POINTER;
+  if (batch < 1 || s_q < 1 || topk < 1 || h_q < 1 || h_q > kMaxRows) return MLA_ERR_BAD_SHAPE;
+  if (static_cast<long long>(batch) * s_q >= (1ll << 30)) return MLA_ERR_BAD_SHAPE;
+  if (h_kv != 1) return MLA_ERR_BAD_HEADS;
+  if (num_sm_parts < 1) return MLA_ERR_BAD_PARTS;
+  const int e = mla::launch_scheduler(nullptr, batch * s_q, num_sm_parts, tile_md, num_splits,
+                                      static_cast<cudaStream_t>(stream), topk);
+  return e == 0 ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_t num_blocks, const int32_t* block_table,
+                              int max_blocks, const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                              int d_v, const int32_t* indices, int topk, const int32_t* tile_md, int num_sm_parts,
+                              const int32_t* num_splits, float softmax_scale, int kv_dtype, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  // ---- argument checks (nothing is enqueued before they all pass) ----
+  if (!q || !kvcache || !block_table || !cache_seqlens || !indices || !tile_md || !num_splits || !out || !lse ||
+      !workspace)
+    return MLA_ERR_NULL_POINTER;
+  if (!aligned(q, 16) || !aligned(kvcache, 16) || !aligned(out, 16) || !aligned(workspace, 16) || !aligned(lse, 4) ||
+      !aligned(indices, 4))
+    return MLA_ERR_MISALIGNED;
+  if (d_v != kDv) return MLA_ERR_BAD_DIM;
+  if (h_kv != 1 || h_q < 1) return MLA_ERR_BAD_HEADS;
+  if (kv_dtype != MLA_KV_BF16) return MLA_ERR_BAD_KV_DTYPE;
+  if (batch < 1 || s_q < 1 || topk < 1 || num_blocks < 1 || max_blocks < 1) return MLA_ERR_BAD_SHAPE;
+  if (h_q > kMaxRows || static_cast<long long>(batch) * s_q >= (1ll << 30)) return MLA_ERR_BAD_SHAPE;
+  if (static_cast<long long>(batch) * s_q * topk >= (1ll << 31)) return MLA_ERR_BAD_SHAPE;
+  if (num_blocks * kPage >= (1ll << 31)) return MLA_ERR_BAD_SHAPE;
+  if (num_sm_parts < 1) return MLA_ERR_BAD_PARTS;
+  const int positions = batch * s_q;
+  const WorkspaceLayout wl = workspace_layout(positions, num_sm_parts, h_q);
+  if (workspace_bytes < wl.total) return MLA_ERR_WORKSPACE;
+
+  EncodeTiledFn encode = encode_fn();
+  if (!encode) return MLA_ERR_CUDA;
+  const int rg = rows_per_cta_for(h_q);
+  // q as {576 dims, h_q heads, batch * s_q positions}; one box = 64 dims x rg heads of a position
+  CUtensorMap tm_q;
+  {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(h_q),
+                          static_cast<cuuint64_t>(positions)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDqk) * 2, static_cast<cuuint64_t>(kDqk) * 2 * h_q};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rg), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  mla::DecodeParams p{};
+  p.block_table = block_table;
+  p.cache_seqlens = cache_seqlens;
+  p.tile_md = tile_md;
+  p.num_splits = num_splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.lse_part = reinterpret_cast<float*>(ws + wl.lse_off);
+  p.o_part = reinterpret_cast<float*>(ws + wl.o_off);
+  p.status = reinterpret_cast<int*>(ws);
+  p.max_blocks = max_blocks;
+  p.batch = positions;  // the scheduler's requests are the query positions
+  p.num_sm_parts = num_sm_parts;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.rows = h_q;
+  p.row_groups = (h_q + rg - 1) / rg;
+  p.causal = 0;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.kv = kvcache;
+  p.indices = indices;
+  p.topk = topk;
+  p.vq = s_q;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int e = mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
+  if (e != 0) return MLA_ERR_CUDA;
+  mla::CombineParams cp{};
+  cp.num_splits = num_splits;
+  cp.o_part = p.o_part;
+  cp.lse_part = p.lse_part;
+  cp.out = p.out;
+  cp.lse = lse;
+  cp.batch = positions;
+  cp.s_q = s_q;
+  cp.h_q = h_q;
+  cp.rows = h_q;
+  cp.vq = s_q;
+  e = mla::launch_combine(cp, st);
+  return e == 0 ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int mla_read_status(void* workspace, int reset, int* status, void* stream) {
   if (!workspace || !status) return MLA_ERR_NULL_POINTER;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

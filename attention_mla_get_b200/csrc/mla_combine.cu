@@ -34,7 +34,9 @@ __global__ void __launch_bounds__(kCombineWarps * 32) mla_combine_kernel(const C
   if (ns == 1 || row >= p.rows) return;
   const int R = p.rows;
   const long long orow = static_cast<long long>(b) * R + row;
-  float* lse_out = p.lse + (static_cast<long long>(b) * p.h_q + row % p.h_q) * p.s_q + row / p.h_q;
+  // token-sparse: request b is query position (b / vq, b % vq) and its rows are the heads
+  float* lse_out = p.vq > 0 ? p.lse + (static_cast<long long>(b / p.vq) * p.h_q + row) * p.vq + b % p.vq
+                            : p.lse + (static_cast<long long>(b) * p.h_q + row % p.h_q) * p.s_q + row / p.h_q;
   __nv_bfloat16* out = p.out + orow * kDv;
   if (ns == 0) {
     for (int d = lane; d < kDv; d += 32) out[d] = __float2bfloat16_rn(0.f);

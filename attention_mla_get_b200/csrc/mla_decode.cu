@@ -128,7 +128,8 @@ struct ChunkWalk {
   }
   __device__ bool next(const DecodeParams& p, int& cb, int& c0, int& c1, int& csplit) {
     while (b < end_b || (b == end_b && blk < end_blk)) {
-      const int n = blocks_of(p.cache_seqlens[b]);
+      // token-sparse: every query position is a request of topk listed positions
+      const int n = blocks_of(p.topk > 0 ? p.topk : p.cache_seqlens[b]);
       const int stop = (b == end_b) ? end_blk : n;
       cb = b;
       c0 = blk;
@@ -238,7 +239,10 @@ __device__ __forceinline__ StepPages step_pages(const int32_t* bt, int st, int n
 // tm_kv is the bf16 cache (64x64 boxes) or, for FP8, the byte view of the cache with 128-byte
 // code boxes; tm_scale (16-byte boxes at byte 512) and tm_rope (128-byte swizzled boxes at byte
 // 528) are used by the FP8 path only.
-template <int RG, bool FP8>
+// SPARSE (bf16 cache only): token-sparse decode.  A "request" b of the chunk walk is the query
+// position (b / vq, b % vq) with topk listed cache positions; the producer warp copies the
+// listed tokens' rows (16-byte cp.async per lane, zeros for empty slots) instead of TMA pages.
+template <int RG, bool FP8, bool SPARSE = false>
 __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                       const __grid_constant__ CUtensorMap tm_scale, const __grid_constant__ CUtensorMap tm_rope,
@@ -271,7 +275,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMaxSlots; ++i) {
-      mbar_init(bar(kBarSlotFull + i), 1);
+      mbar_init(bar(kBarSlotFull + i), SPARSE ? 32 : 1);  // SPARSE: one cp.async arrival per lane
       mbar_init(bar(kBarSlotEmpty + i), 1);
     }
     for (int i = 0; i < kNumS; ++i) {
@@ -317,7 +321,75 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
 
   pdl_launch_dependents();
 
-  if (warp == 4) {
+  if (SPARSE && warp == 4) {
+    // ======================== gather producer (token-sparse) =======================
+    // Each lane copies token rows lane, lane + 32, lane + 64, lane + 96 of a step: for every
+    // 64-dim column of the slot, eight 16-byte cp.async into the row's swizzled chunks.  The
+    // slot's full barrier counts one arrival per lane, made when that lane's copies landed.
+    uint32_t g = 0;
+    int q_fills = 0;
+    bool ok = true;
+    const char* kvb = static_cast<const char*>(p.kv);
+    long long rowoff[4];  // byte offset of each of this lane's token rows (-1: empty slot)
+    ChunkWalk walk(p, part);
+    int b, c0, c1, split;
+    while (ok && walk.next(p, b, c0, c1, split)) {
+      const int breal = b / p.vq;
+      const int L = p.cache_seqlens[breal];
+      const int32_t* bt = p.block_table + static_cast<long long>(breal) * p.max_blocks;
+      const int32_t* ind = p.indices + static_cast<long long>(b) * p.topk;
+      if (lane == 0) {
+        ok = mbar_wait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc);
+        if (ok) {
+          mbar_arrive_expect_tx(bar(kBarQFull), 9u * C::kQAtomBytes);
+          for (int a = 0; a < 9; ++a) tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, 64 * a, rg * RG, b, bar(kBarQFull));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      ++q_fills;
+      const int n = c1 - c0;
+      auto rows_of = [&](int t) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int pos = (c0 + t) * kBlockTokens + lane + 32 * k;
+          const int idx = pos < p.topk ? ind[pos] : -1;
+          rowoff[k] = (idx >= 0 && idx < L)
+                          ? (static_cast<long long>(bt[idx >> 6]) * kPage + (idx & (kPage - 1))) * (kDqk * 2)
+                          : -1;
+        }
+      };
+      auto fill = [&](int dims0, int natoms) -> bool {
+        const int s = static_cast<int>(g % C::kNumSlots);
+        const uint32_t use = g / C::kNumSlots;
+        if (!warp_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc, lane)) return false;
+        const uint32_t dst = sSlots + static_cast<uint32_t>(s) * C::kSlotBytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t r = static_cast<uint32_t>(lane + 32 * k);
+          const bool valid = rowoff[k] >= 0;
+          const char* src = kvb + (valid ? rowoff[k] : 0) + dims0 * 2;
+          for (int a = 0; a < natoms; ++a)
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              cp_async_16(dst + a * C::kAtomColBytes + r * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4),
+                          src + (64 * a + 8 * c) * 2, valid ? 16u : 0u);
+        }
+        cp_async_arrive_noinc(bar(kBarSlotFull + s));
+        ++g;
+        return true;
+      };
+      for (int e = 0; ok && e < order_len(n); ++e) {
+        bool is_v;
+        int t;
+        order_at(e, n, is_v, t);
+        rows_of(t);
+        for (int ks = 0; ok && ks < 4; ++ks) ok = fill(128 * ks, 2);
+        if (ok && !is_v) ok = fill(kDv, 1);
+      }
+    }
+    cp_async_wait_all();  // this lane's copies have landed before the CTA may exit
+  } else if (warp == 4) {
     // ================================ TMA producer ================================
     if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();
@@ -429,6 +501,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
         s = g % C::kNumSlots;
         if (!mbar_wait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) return false;
         ++g;
+        if (SPARSE) fence_proxy_async_smem();  // slots written by cp.async (generic proxy)
         tc_fence_after();
         return true;
       };
@@ -517,7 +590,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
     ChunkWalk walk(p, part);
     int b, c0, c1, split;
     while (walk.next(p, b, c0, c1, split)) {
-      const int L = p.cache_seqlens[b];
+      const int L = p.cache_seqlens[SPARSE ? b / p.vq : b];
       const int n = c1 - c0;
       const bool single = (p.num_splits[b + 1] - p.num_splits[b]) == 1;
       const int row0 = rg * RG;
@@ -539,11 +612,17 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
         // j <= L - s_q + r / h_q (the query block sits at the end of the cache).  With
         // i0 = j - L + s_q that is r / h_q >= i0, i.e. r >= i0 * h_q, i.e. c >= cmin.
         int cmin = -(1 << 30);
-        if (p.causal) {
-          const int i0 = j - L + p.s_q;
-          if (i0 > 0) cmin = i0 * p.h_q - row0;
+        if constexpr (SPARSE) {
+          // token-sparse: slot j of the list is a key iff it names a position in [0, L)
+          const int idx = j < p.topk ? p.indices[static_cast<long long>(b) * p.topk + j] : -1;
+          if (idx < 0 || idx >= L) cmin = 1 << 30;
+        } else {
+          if (p.causal) {
+            const int i0 = j - L + p.s_q;
+            if (i0 > 0) cmin = i0 * p.h_q - row0;
+          }
+          if (j >= L) cmin = 1 << 30;
         }
-        if (j >= L) cmin = 1 << 30;
 #pragma unroll
         for (int c = 0; c < RG; ++c) x[c] = (c >= cmin) ? x[c] * p.scale_log2 : NEG_INF;
         float v[RG];
@@ -616,7 +695,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
           }
           tmem_wait_st();
         }
-        if (!FP8 && t0 + kBlockTokens > L) {
+        if (!FP8 && !SPARSE && t0 + kBlockTokens > L) {
           // tail step: zero the V rows of tokens past the end (their cache slots may hold NaN,
           // and 0 * NaN would poison O)
           for (int vs = 0; vs < 4; ++vs) {
@@ -650,10 +729,14 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
         const float lse_val = l > 0.f ? (m_ref + log2f(l)) * kLn2 : NEG_INF;
         inv_sm[tid] = l > 0.f ? 1.f / l : 0.f;
         if (row < R) {
-          if (single)
-            p.lse[(static_cast<long long>(b) * p.h_q + row % p.h_q) * p.s_q + row / p.h_q] = lse_val;
-          else
+          if (single) {
+            if (SPARSE)  // query position (b / vq, b % vq), head row
+              p.lse[(static_cast<long long>(b / p.vq) * p.h_q + row) * p.vq + b % p.vq] = lse_val;
+            else
+              p.lse[(static_cast<long long>(b) * p.h_q + row % p.h_q) * p.s_q + row / p.h_q] = lse_val;
+          } else {
             p.lse_part[static_cast<long long>(split) * R + row] = lse_val;
+          }
         }
         m_ref = NEG_INF;
       }
@@ -804,11 +887,11 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
   }
 }
 
-template <int RG, bool FP8>
+template <int RG, bool FP8, bool SPARSE = false>
 int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_scale,
                 const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
   using C = Cfg<RG, FP8>;
-  auto kern = mla_decode_kernel<RG, FP8>;
+  auto kern = mla_decode_kernel<RG, FP8, SPARSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid(p.num_sm_parts, p.row_groups, 1);
@@ -824,6 +907,15 @@ int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const 
     case 16: return launch_impl<16, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
     case 32: return launch_impl<32, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
     case 64: return launch_impl<64, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+    default: return static_cast<int>(cudaErrorInvalidValue);
+  }
+}
+
+int launch_decode_sparse_bf16(const CUtensorMap& tm_q, const DecodeParams& p, int rows_per_cta, cudaStream_t stream) {
+  switch (rows_per_cta) {
+    case 16: return launch_impl<16, false, true>(tm_q, tm_q, tm_q, tm_q, p, stream);
+    case 32: return launch_impl<32, false, true>(tm_q, tm_q, tm_q, tm_q, p, stream);
+    case 64: return launch_impl<64, false, true>(tm_q, tm_q, tm_q, tm_q, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }
 }

@@ -40,6 +40,12 @@ struct DecodeParams {
   int row_groups;         // G = ceil(R / rows per CTA, or per CTA pair)
   int causal;
   float scale_log2;       // softmax_scale * log2(e)
+  // token-sparse decode (topk > 0): the scheduler's "requests" are the batch * s_q query
+  // positions (vq = s_q of them per request), each over topk listed cache positions
+  const void* kv;         // the bf16 cache (read with per-token copies)
+  const int32_t* indices; // [batch * s_q, topk] logical cache positions; others: empty slots
+  int topk;
+  int vq;
 };
 
 struct CombineParams {
@@ -52,6 +58,7 @@ struct CombineParams {
   int s_q;
   int h_q;
   int rows;
+  int vq;  // token-sparse: query positions per request (batch counts positions), else 0
 };
 
 inline int row_groups_for(int rows) { return rows <= kRowsPerCta ? 1 : (rows + kRowsPerCta - 1) / kRowsPerCta; }
@@ -63,12 +70,14 @@ inline bool use_pair_kernel(int rows, bool /*fp8*/) { return rows > kRowsPerCta;
 inline int sms_per_part(int rows) { return rows <= kRowsPerCta ? 1 : 2 * ((rows + kPairRows - 1) / kPairRows); }
 
 // launchers (return cudaError_t as int)
+// cache_seqlens == nullptr: every one of the `batch` requests has uniform_len tokens
 int launch_scheduler(const int32_t* cache_seqlens, int batch, int num_sm_parts, int32_t* tile_md,
-                     int32_t* num_splits, cudaStream_t stream);
+                     int32_t* num_splits, cudaStream_t stream, int uniform_len = 0);
 int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, int rows_per_cta,
                        cudaStream_t stream);
 int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
                       const CUtensorMap& tm_rope, const DecodeParams& p, int rows_per_cta, cudaStream_t stream);
+int launch_decode_sparse_bf16(const CUtensorMap& tm_q, const DecodeParams& p, int rows_per_cta, cudaStream_t stream);
 int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
                             cudaStream_t stream);
 int launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,

@@ -54,8 +54,10 @@ __device__ long long block_scan(long long v, long long* warp_tot, long long* tot
 }
 
 __global__ void __launch_bounds__(kSchedThreads)
-    mla_tile_scheduler_kernel(const int32_t* __restrict__ seqlens, int batch, int parts, int32_t* __restrict__ md,
-                              int32_t* __restrict__ ns) {
+    mla_tile_scheduler_kernel(const int32_t* __restrict__ seqlens, int uniform_len, int batch, int parts,
+                              int32_t* __restrict__ md, int32_t* __restrict__ ns) {
+  // seqlens == nullptr: every request has uniform_len tokens (token-sparse decode: the
+  // requests are the query positions, each over its topk listed positions)
   __shared__ long long warp_tot[32];
   __shared__ int32_t s_cum[kSmemBatch + 1];  // C_{b+1}: binary searches stay on chip
   const long long F = kFixedSplitCost;
@@ -66,7 +68,7 @@ __global__ void __launch_bounds__(kSchedThreads)
   long long carry = 0;
   for (int base = 0; base < batch; base += kSchedThreads) {
     const int b = base + tid;
-    const long long n = b < batch ? blocks_of(seqlens[b]) : 0;
+    const long long n = b < batch ? blocks_of(seqlens ? seqlens[b] : uniform_len) : 0;
     long long tile_total;
     const long long incl = block_scan(n > 0 ? n + F : 0, warp_tot, &tile_total) + carry;
     if (b < batch) {
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(kSchedThreads)
   long long chunk_carry = 0;
   for (int base = 0; base < batch; base += kSchedThreads) {
     const int b = base + tid;
-    const long long n = b < batch ? blocks_of(seqlens[b]) : 0;
+    const long long n = b < batch ? blocks_of(seqlens ? seqlens[b] : uniform_len) : 0;
     long long tile_total;
     const long long incl = block_scan(n > 0 ? n + F : 0, warp_tot, &tile_total) + carry;
     const long long cb = incl - (n > 0 ? n + F : 0);
@@ -149,9 +151,9 @@ __global__ void __launch_bounds__(kSchedThreads)
 }  // namespace
 
 int launch_scheduler(const int32_t* cache_seqlens, int batch, int num_sm_parts, int32_t* tile_md,
-                     int32_t* num_splits, cudaStream_t stream) {
-  mla_tile_scheduler_kernel<<<1, kSchedThreads, 0, stream>>>(cache_seqlens, batch, num_sm_parts, tile_md,
-                                                             num_splits);
+                     int32_t* num_splits, cudaStream_t stream, int uniform_len) {
+  mla_tile_scheduler_kernel<<<1, kSchedThreads, 0, stream>>>(cache_seqlens, uniform_len, batch, num_sm_parts,
+                                                             tile_md, num_splits);
   return static_cast<int>(cudaGetLastError());
 }
 

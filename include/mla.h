@@ -152,6 +152,34 @@ MLA_API int mla_decode_kvcache_noalloc(const void* q, const void* kvcache, int64
                                        int kv_dtype, void* out, float* lse, void* stream);
 
 /*
+ * Token-sparse decode (the `topk` argument of get_mla_metadata and the `indices` argument of
+ * flash_mla_with_kvcache on the gitcode FlashMLA page, "解码阶段使用示例" / "稀疏解码场景").
+ * The page names the arguments but not their shape; this library's reading:
+ *   indices        device int32 [batch, s_q, topk], 4-byte aligned: query position i of
+ *                  request b attends to the tokens at the logical cache positions
+ *                  indices[b, i, :] (through block_table, as in dense decode).  An entry
+ *                  outside [0, cache_seqlens[b]) is an empty slot; a position listed twice
+ *                  counts twice.  No causal mask applies.  A query with no valid entry gets
+ *                  O = 0 and LSE = -inf.
+ * Every query position is scheduled as a request of topk tokens:
+ *   mla_get_metadata_sparse  tile_md [num_sm_parts, 8] and num_splits [batch * s_q + 1] for
+ *                            batch * s_q positions of topk tokens; num_sm_parts from
+ *                            mla_num_sm_parts(h_q, h_kv)
+ *   mla_decode_kvcache_sparse  as mla_decode_kvcache (bf16 cache only: MLA_ERR_BAD_KV_DTYPE
+ *                            otherwise), with the workspace of
+ *                            mla_workspace_size(batch * s_q, num_sm_parts, h_q, h_kv) bytes
+ */
+MLA_API int mla_get_metadata_sparse(int batch, int s_q, int topk, int h_q, int h_kv, int32_t* tile_md,
+                                    int num_sm_parts, int32_t* num_splits, void* stream);
+
+MLA_API int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_t num_blocks,
+                                      const int32_t* block_table, int max_blocks, const int32_t* cache_seqlens,
+                                      int batch, int s_q, int h_q, int h_kv, int d_v, const int32_t* indices,
+                                      int topk, const int32_t* tile_md, int num_sm_parts,
+                                      const int32_t* num_splits, float softmax_scale, int kv_dtype, void* out,
+                                      float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Reads the device status word of a workspace into *status (host pointer).  This call
  * synchronises `stream`.  reset != 0 clears the word afterwards (enqueued on `stream`).
  */

@@ -56,3 +56,20 @@ def compare(case, out, lse, O_ref, L_ref, requests=None, fp8=None):
     worst_l = float(dl.max()) if dl.size else 0.0
     assert worst_l <= l_tol, f"LSE out of tolerance: max |dLSE| = {worst_l:.3e}"
     return {"max_dO": worst_o, "max_dLSE": worst_l}
+
+
+def run_gpu_sparse(case: mi.DecodeCase, indices, num_sm_parts=None, tensors=None):
+    """Token-sparse decode of `case` over `indices` (int32 [b, s_q, topk]) through the library."""
+    import attention_mla_get_b200 as mla
+    q, kv, bt, sl = tensors if tensors is not None else to_device(case)
+    idx = torch.from_numpy(np.ascontiguousarray(indices, dtype=np.int32)).to(q.device)
+    topk = idx.shape[-1]
+    md, ns = mla.mla_get_metadata_sparse(case.batch, case.s_q, topk, case.h_q, 1, num_sm_parts=num_sm_parts,
+                                         device=q.device)
+    ws = torch.zeros(mla.mla_workspace_size(case.batch * case.s_q, md.shape[0], case.h_q, 1), dtype=torch.uint8,
+                     device=q.device)
+    out, lse = mla.mla_decode_kvcache_sparse(q, kv, bt, sl, idx, 512, md, ns, softmax_scale=case.softmax_scale,
+                                             workspace=ws)
+    torch.cuda.synchronize()
+    status = mla.mla_read_status(ws)
+    return out.float().cpu().numpy(), lse.cpu().numpy(), status, (md, ns)

@@ -38,7 +38,8 @@ def _declared():
 def test_every_declared_symbol_is_exported(lib):
     names = _declared()
     assert set(names) == {"mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-                          "mla_decode_kvcache_noalloc", "mla_read_status", "mla_strerror", "mla_version"}
+                          "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
+                          "mla_read_status", "mla_strerror", "mla_version"}
     so = os.path.join(ROOT, "attention_mla_get_b200", "libmla.so")
     nm = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True).stdout
     exported = set(re.findall(r" T (mla_\w+)", nm))
@@ -106,3 +107,39 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert lib.mla_get_metadata(fake, 0, 16, 1, fake, 4, fake, None) == -7
     assert lib.mla_get_metadata(fake, 2, 16, 2, fake, 4, fake, None) == -4
     assert lib.mla_get_metadata(fake, 2, 16, 1, fake, 0, fake, None) == -8
+
+
+def _call_sparse(lib, **kw):
+    """mla_decode_kvcache_sparse with plausible fake pointers (never dereferenced: every case
+    below fails an argument check before anything is enqueued)."""
+    fake = ctypes.c_void_p(0x10000)
+    a = dict(q=fake, kv=fake, nb=8, bt=fake, mb=4, sl=fake, b=2, s_q=1, h_q=16, h_kv=1, d_v=512, idx=fake,
+             topk=64, md=fake, parts=4, ns=fake, scale=0.04, dt=0, out=fake, lse=fake, ws=fake, wsb=1 << 30)
+    a.update(kw)
+    f = lib.mla_decode_kvcache_sparse
+    i32, i64, vp, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+    f.argtypes = [vp, vp, i64, vp, i32, vp, i32, i32, i32, i32, i32, vp, i32, vp, i32, vp, ctypes.c_float, i32,
+                  vp, vp, vp, sz, vp]
+    f.restype = i32
+    return f(a["q"], a["kv"], a["nb"], a["bt"], a["mb"], a["sl"], a["b"], a["s_q"], a["h_q"], a["h_kv"], a["d_v"],
+             a["idx"], a["topk"], a["md"], a["parts"], a["ns"], a["scale"], a["dt"], a["out"], a["lse"], a["ws"],
+             a["wsb"], None)
+
+
+def test_sparse_argument_errors_are_reported_before_any_launch(lib):
+    assert _call_sparse(lib, idx=None) == -1
+    assert _call_sparse(lib, idx=ctypes.c_void_p(0x10002)) == -2
+    assert _call_sparse(lib, d_v=256) == -3
+    assert _call_sparse(lib, h_kv=2) == -4
+    assert _call_sparse(lib, dt=1) == -5             # token-sparse decode reads bf16 caches only
+    assert _call_sparse(lib, topk=0) == -7
+    assert _call_sparse(lib, s_q=0) == -7
+    assert _call_sparse(lib, parts=0) == -8
+    assert _call_sparse(lib, wsb=100) == -6
+    fake = ctypes.c_void_p(0x10000)
+    g = lib.mla_get_metadata_sparse
+    g.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    assert g(2, 1, 64, 16, 1, None, 4, fake, None) == -1
+    assert g(2, 1, 0, 16, 1, fake, 4, fake, None) == -7
+    assert g(2, 1, 64, 16, 2, fake, 4, fake, None) == -4
+    assert g(2, 1, 64, 16, 1, fake, 0, fake, None) == -8
