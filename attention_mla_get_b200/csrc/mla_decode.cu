@@ -78,7 +78,7 @@ struct Cfg {
   static constexpr int kOffRaw = kOffSlots + kNumSlots * kSlotBytes;
   static constexpr int kOffScale = kOffRaw + kNumRaw * kRawBytes;
   static constexpr int kOffMisc = kOffScale + kNumScale * kScaleBytes;
-  static constexpr int kMiscBytes = 3072;
+  static constexpr int kMiscBytes = 3584;  // + 512 B: token-sparse row table
   static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
   static constexpr uint32_t kPSwzMask = RG / 8 - 1;                // (row bytes / 16) - 1
   static constexpr uint32_t kPLayout = RG == 64 ? kSwizzle128 : (RG == 32 ? kSwizzle64 : kSwizzle32);
@@ -264,6 +264,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
   float* m_sm = reinterpret_cast<float*>(misc + 2048);      // [64]
   float* alpha_sm = reinterpret_cast<float*>(misc + 2304);  // [64]
   float* inv_sm = reinterpret_cast<float*>(misc + 2560);    // [64]
+  int32_t* row_tab = reinterpret_cast<int32_t*>(misc + 3072);  // [128] SPARSE: cache row per token slot
   static_assert(kNumBars * 8 <= 512, "barrier area");
   auto bar = [&](int i) -> uint32_t { return sBars + 8u * static_cast<uint32_t>(i); };
 
@@ -323,14 +324,14 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
 
   if (SPARSE && warp == 4) {
     // ======================== gather producer (token-sparse) =======================
-    // Each lane copies token rows lane, lane + 32, lane + 64, lane + 96 of a step: for every
-    // 64-dim column of the slot, eight 16-byte cp.async into the row's swizzled chunks.  The
+    // The 128 listed tokens of a step are looked up once per step group (row_tab: physical cache
+    // row, -1 for an empty slot); then every warp-wide cp.async copies whole 16-byte chunks of
+    // two (or four) token rows, so each instruction reads a few contiguous row segments.  The
     // slot's full barrier counts one arrival per lane, made when that lane's copies landed.
     uint32_t g = 0;
     int q_fills = 0;
     bool ok = true;
     const char* kvb = static_cast<const char*>(p.kv);
-    long long rowoff[4];  // byte offset of each of this lane's token rows (-1: empty slot)
     ChunkWalk walk(p, part);
     int b, c0, c1, split;
     while (ok && walk.next(p, b, c0, c1, split)) {
@@ -350,30 +351,32 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
       ++q_fills;
       const int n = c1 - c0;
       auto rows_of = [&](int t) {
+        __syncwarp();  // the previous group's copies were all issued
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int pos = (c0 + t) * kBlockTokens + lane + 32 * k;
+          const int r = lane + 32 * k;
+          const int pos = (c0 + t) * kBlockTokens + r;
           const int idx = pos < p.topk ? ind[pos] : -1;
-          rowoff[k] = (idx >= 0 && idx < L)
-                          ? (static_cast<long long>(bt[idx >> 6]) * kPage + (idx & (kPage - 1))) * (kDqk * 2)
-                          : -1;
+          row_tab[r] = (idx >= 0 && idx < L) ? bt[idx >> 6] * kPage + (idx & (kPage - 1)) : -1;
         }
+        __syncwarp();
       };
+      // natoms 64-dim columns from dims0: a row slice is 16 * natoms chunks of 16 bytes
       auto fill = [&](int dims0, int natoms) -> bool {
         const int s = static_cast<int>(g % C::kNumSlots);
         const uint32_t use = g / C::kNumSlots;
         if (!warp_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc, lane)) return false;
         const uint32_t dst = sSlots + static_cast<uint32_t>(s) * C::kSlotBytes;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t r = static_cast<uint32_t>(lane + 32 * k);
-          const bool valid = rowoff[k] >= 0;
-          const char* src = kvb + (valid ? rowoff[k] : 0) + dims0 * 2;
-          for (int a = 0; a < natoms; ++a)
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              cp_async_16(dst + a * C::kAtomColBytes + r * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4),
-                          src + (64 * a + 8 * c) * 2, valid ? 16u : 0u);
+        const int cpr = 8 * natoms;        // chunks per row slice
+        const int rpi = 32 / cpr;          // rows per warp instruction
+        const int sub = lane / cpr, c = lane % cpr;
+        const uint32_t a = static_cast<uint32_t>(c >> 3), cc = static_cast<uint32_t>(c & 7);
+        const char* src0 = kvb + (dims0 + 8 * c) * 2;
+        for (int i = 0; i < kBlockTokens / rpi; ++i) {
+          const uint32_t r = static_cast<uint32_t>(i * rpi + sub);
+          const int row = row_tab[r];
+          cp_async_16(dst + a * C::kAtomColBytes + r * 128u + ((cc ^ (r & 7u)) << 4),
+                      src0 + (row >= 0 ? static_cast<long long>(row) * (kDqk * 2) : 0), row >= 0 ? 16u : 0u);
         }
         cp_async_arrive_noinc(bar(kBarSlotFull + s));
         ++g;

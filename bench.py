@@ -123,13 +123,17 @@ def oracle_baseline(case, budget_s: float = 15.0):
     t0 = time.perf_counter()
     done = []
     for b in range(case.batch):
-        oracle.mla_decode_reference(case, requests=[b])
+        if case.indices is not None:
+            oracle.mla_sparse_decode_reference(case, case.indices, requests=[b])
+        else:
+            oracle.mla_decode_reference(case, requests=[b])
         done.append(b)
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
     sub = mi.DecodeCase(**{**case.__dict__, "cache_seqlens": case.cache_seqlens[done],
-                           "q_bits": case.q_bits[done], "block_table": case.block_table[done]})
+                           "q_bits": case.q_bits[done], "block_table": case.block_table[done],
+                           "indices": None if case.indices is None else case.indices[done]})
     units = mi.workload_units(sub)
     try:
         from threadpoolctl import threadpool_info
@@ -152,8 +156,11 @@ def rank_case(workload: str, rank: int, batch=None):
     w = mi.WORKLOADS[workload]
     case = mi.make_workload(workload, poison=False, batch=batch)
     if rank > 0:
+        idx = case.indices
         case = mi.make_case(case.batch, case.s_q, case.h_q, case.cache_seqlens, causal=case.causal,
                             kv_format=case.kv_format, seed=w.seed + 1000 * rank, poison=False, name=workload)
+        if idx is not None:
+            case.indices = mi.make_sparse_indices(case.cache_seqlens, case.s_q, w.topk, w.seed + 1000 * rank)
     return case
 
 
@@ -209,7 +216,8 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(timed),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": args.workload, "batch": w.batch, "s_q": w.s_q,
-                                                 "h_q": w.h_q, "seqlens": w.seqlens, "kv": w.kv_format},
+                                                 "h_q": w.h_q, "seqlens": w.seqlens, "kv": w.kv_format,
+                                                 "topk": w.topk},
                 "cpu_baseline": {"value": value, "unit": "GB/s", "cores": timed[0]["cores"], "kind": "oracle",
                                  "sample": f"first {timed[0]['requests']} of {w.batch} requests per step"},
                 "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -237,17 +245,34 @@ def main():
     case = rank_case(args.workload, rank, args.batch)
     units = mi.workload_units(case)
     q, kv, bt, sl = to_device(case, dev)
+    sparse = case.indices is not None
+    idx = torch.from_numpy(case.indices).to(dev) if sparse else None
     R = case.rows
-    parts = mla.mla_num_sm_parts(R, 1, local)
-    ws = torch.zeros(mla.mla_workspace_size(case.batch, parts, R, 1), dtype=torch.uint8, device=dev)
+    # token-sparse: the scheduler's requests are the batch * s_q query positions of h_q rows
+    parts = mla.mla_num_sm_parts(case.h_q if sparse else R, 1, local)
+    ws = torch.zeros(mla.mla_workspace_size(case.batch * case.s_q, parts, case.h_q, 1) if sparse else
+                     mla.mla_workspace_size(case.batch, parts, R, 1), dtype=torch.uint8, device=dev)
     out = torch.empty((case.batch, case.s_q, case.h_q, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((case.batch, case.h_q, case.s_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def metadata(sl_):
+        if sparse:
+            return mla.mla_get_metadata_sparse(case.batch, case.s_q, case.topk, case.h_q, 1, num_sm_parts=parts,
+                                               device=dev)
+        return mla.mla_get_metadata(sl_, R, 1, num_sm_parts=parts)
+
+    def decode(q_, bt_, sl_, idx_, md, ns):
+        if sparse:
+            mla.mla_decode_kvcache_sparse(q_, kv, bt_, sl_, idx_, 512, md, ns, softmax_scale=case.softmax_scale,
+                                          out=out, lse=lse, workspace=ws)
+        else:
+            mla.mla_decode_kvcache(q_, kv, bt_, sl_, 512, md, ns, softmax_scale=case.softmax_scale,
+                                   causal=case.causal, out=out, lse=lse, workspace=ws)
+
     def step():
-        md, ns = mla.mla_get_metadata(sl, R, 1, num_sm_parts=parts)
-        mla.mla_decode_kvcache(q, kv, bt, sl, 512, md, ns, softmax_scale=case.softmax_scale, causal=case.causal,
-                               out=out, lse=lse, workspace=ws)
+        md, ns = metadata(sl)
+        decode(q, bt, sl, idx, md, ns)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -260,7 +285,7 @@ def main():
     barrier()
 
     # ---- device-timed steps, with per-call events for the decode kernel's roofline ----
-    md0, ns0 = mla.mla_get_metadata(sl, R, 1, num_sm_parts=parts)
+    md0, ns0 = metadata(sl)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -268,10 +293,9 @@ def main():
         t_wall0 = time.perf_counter()
         start.record(stream)
         for i in range(args.steps):
-            md, ns = mla.mla_get_metadata(sl, R, 1, num_sm_parts=parts)
+            md, ns = metadata(sl)
             ev[i][0].record(stream)
-            mla.mla_decode_kvcache(q, kv, bt, sl, 512, md, ns, softmax_scale=case.softmax_scale,
-                                   causal=case.causal, out=out, lse=lse, workspace=ws)
+            decode(q, bt, sl, idx, md, ns)
             ev[i][1].record(stream)
         stop.record(stream)
         barrier()
@@ -287,16 +311,19 @@ def main():
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     q_d, bt_d, sl_d = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(sl)
-    h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
+    idx_h = idx.cpu().pin_memory() if sparse else None
+    idx_d = torch.empty_like(idx) if sparse else None
+    h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4 + (idx_h.numel() * 4 if sparse else 0)
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
 
     def e2e_step():
         q_d.copy_(q_h, non_blocking=True)
         bt_d.copy_(bt_h, non_blocking=True)
         sl_d.copy_(sl_h, non_blocking=True)
-        md, ns = mla.mla_get_metadata(sl_d, R, 1, num_sm_parts=parts)
-        mla.mla_decode_kvcache(q_d, kv, bt_d, sl_d, 512, md, ns, softmax_scale=case.softmax_scale,
-                               causal=case.causal, out=out, lse=lse, workspace=ws)
+        if sparse:
+            idx_d.copy_(idx_h, non_blocking=True)
+        md, ns = metadata(sl_d)
+        decode(q_d, bt_d, sl_d, idx_d, md, ns)
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
 
@@ -336,6 +363,7 @@ def main():
         "dtype": "f16" if case.kv_format == "fp8" and case.s_q * case.h_q > 64 else "bf16",
         "config": {"workload": args.workload, "batch": case.batch, "s_q": case.s_q, "h_q": case.h_q,
                    "h_kv": 1, "d_qk": 576, "d_v": 512, "page": 64, "seqlens": w.seqlens, "causal": case.causal,
+                   "topk": case.topk,
                    "kv": case.kv_format, "kv_bytes": units["kv_bytes"], "l2": "inputs larger than L2 (no flush)",
                    "parallelism": f"replicas x{world} (independent requests per GPU)"},
         "tflops": tflops,
