@@ -74,6 +74,9 @@ def _load() -> ctypes.CDLL:
     lib.mla_decode_kvcache_sparse.argtypes = [vp, vp, i64, vp, i32, vp, i32, i32, i32, i32, i32, vp, i32, vp, i32,
                                               vp, ctypes.c_float, i32, vp, vp, vp, sz, vp]
     lib.mla_decode_kvcache_sparse.restype = i32
+    lib.mla_sparse_prefill.argtypes = [vp, vp, i32, vp, i32, i32, i32, i32, i32, vp, i32, vp, ctypes.c_float, vp, vp,
+                                       vp, sz, vp]
+    lib.mla_sparse_prefill.restype = i32
     lib.mla_read_status.argtypes = [vp, i32, ctypes.POINTER(i32), vp]
     lib.mla_read_status.restype = i32
     lib.mla_strerror.argtypes = [i32]
@@ -86,7 +89,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 
 EXPORTED = ("mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-            "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
+            "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse", "mla_sparse_prefill",
             "mla_read_status", "mla_strerror", "mla_version")
 
 
@@ -247,6 +250,46 @@ def mla_decode_kvcache_sparse(q: torch.Tensor, kvcache: torch.Tensor, block_tabl
     return out, lse
 
 
+def mla_sparse_prefill(q: torch.Tensor, kv: torch.Tensor, indices: torch.Tensor, softmax_scale: float,
+                       d_v: int = D_V, tile_md: Optional[torch.Tensor] = None, num_splits: Optional[torch.Tensor] = None,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Sparse prefill: q bf16 [s_q, h_q, 576], kv bf16 [s_kv, (1,) 576], indices int32 [s_q, (1,) topk]
+    -> (out bf16 [s_q, h_q, 512], lse fp32 [h_q, s_q]).  Metadata is computed when not given."""
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[-1] != D_QK:
+        raise ValueError("q must be bf16 [s_q, h_q, 576]")
+    q = q.contiguous()
+    s_q, h_q, _ = q.shape
+    if kv.dtype != torch.bfloat16 or kv.shape[-1] != D_QK or not kv.is_contiguous():
+        raise ValueError("kv must be contiguous bf16 [s_kv, (1,) 576]")
+    s_kv = kv.shape[0]
+    idx = indices.reshape(s_q, -1) if indices.dim() == 3 else indices
+    if idx.dtype != torch.int32 or idx.dim() != 2 or idx.shape[0] != s_q:
+        raise ValueError("indices must be int32 [s_q, (1,) topk]")
+    idx = idx.contiguous()
+    topk = idx.shape[1]
+    if tile_md is None or num_splits is None:
+        tile_md, num_splits = mla_get_metadata_sparse(1, s_q, topk, h_q, 1, device=q.device, stream=stream)
+    num_sm_parts = tile_md.shape[0]
+    if out is None:
+        out = torch.empty((s_q, h_q, D_V), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((h_q, s_q), dtype=torch.float32, device=q.device)
+    need = mla_workspace_size(s_q, num_sm_parts, h_q, 1)
+    if workspace is None:
+        workspace = torch.zeros((max(need, 256),), dtype=torch.uint8, device=q.device)
+    _check(_lib.mla_sparse_prefill(_ptr(q), _ptr(kv), int(s_kv), _ptr(idx), int(s_q), int(h_q), 1, int(d_v),
+                                   int(topk), _ptr(tile_md), num_sm_parts, _ptr(num_splits), float(softmax_scale),
+                                   _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "mla_sparse_prefill")
+    return out, lse
+
+
+def flash_mla_sparse_fwd(q, kv, indices, sm_scale, d_v=D_V):
+    """The spelling of the sparse prefill call on the pages."""
+    return mla_sparse_prefill(q, kv, indices, sm_scale, d_v=d_v)
+
+
 def mla_read_status(workspace: torch.Tensor, reset: bool = False, stream=None) -> int:
     v = ctypes.c_int(0)
     _check(_lib.mla_read_status(_ptr(workspace), 1 if reset else 0, ctypes.byref(v), _stream(stream)),
@@ -268,7 +311,7 @@ def flash_mla_with_kvcache(q, k_cache, block_table, cache_seqlens, head_dim_v, t
 
 __all__ = [
     "mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache", "mla_read_status",
-    "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
+    "mla_get_metadata_sparse", "mla_decode_kvcache_sparse", "mla_sparse_prefill", "flash_mla_sparse_fwd",
     "mla_strerror", "mla_version", "get_mla_metadata", "flash_mla_with_kvcache", "MLAError", "LIB_PATH",
     "KV_BF16", "KV_FP8",
 ]

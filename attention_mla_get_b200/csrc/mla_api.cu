@@ -308,6 +308,77 @@ int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_t num_bl
   return e == 0 ? MLA_OK : MLA_ERR_CUDA;
 }
 
+int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const int32_t* indices, int s_q, int h_q, int h_kv,
+                       int d_v, int topk, const int32_t* tile_md, int num_sm_parts, const int32_t* num_splits,
+                       float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (!q || !kv || !indices || !tile_md || !num_splits || !out || !lse || !workspace) return MLA_ERR_NULL_POINTER;
+  if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(workspace, 16) || !aligned(lse, 4) ||
+      !aligned(indices, 4))
+    return MLA_ERR_MISALIGNED;
+  if (d_v != kDv) return MLA_ERR_BAD_DIM;
+  if (h_kv != 1 || h_q < 1) return MLA_ERR_BAD_HEADS;
+  if (s_kv < 1 || s_q < 1 || topk < 1 || h_q > kMaxRows || s_q >= (1 << 30)) return MLA_ERR_BAD_SHAPE;
+  if (static_cast<long long>(s_q) * topk >= (1ll << 31)) return MLA_ERR_BAD_SHAPE;
+  if (num_sm_parts < 1) return MLA_ERR_BAD_PARTS;
+  const WorkspaceLayout wl = workspace_layout(s_q, num_sm_parts, h_q);
+  if (workspace_bytes < wl.total) return MLA_ERR_WORKSPACE;
+  EncodeTiledFn encode = encode_fn();
+  if (!encode) return MLA_ERR_CUDA;
+  const int rg = rows_per_cta_for(h_q);
+  CUtensorMap tm_q;  // {576 dims, h_q heads, s_q query tokens}
+  {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(h_q), static_cast<cuuint64_t>(s_q)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDqk) * 2, static_cast<cuuint64_t>(kDqk) * 2 * h_q};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rg), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (encode(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  mla::DecodeParams p{};
+  p.block_table = nullptr;  // the cache is contiguous: logical position = row
+  p.cache_seqlens = nullptr;
+  p.kv_len = s_kv;
+  p.tile_md = tile_md;
+  p.num_splits = num_splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.lse_part = reinterpret_cast<float*>(ws + wl.lse_off);
+  p.o_part = reinterpret_cast<float*>(ws + wl.o_off);
+  p.status = reinterpret_cast<int*>(ws);
+  p.batch = s_q;  // one request of s_q query positions
+  p.num_sm_parts = num_sm_parts;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.rows = h_q;
+  p.row_groups = (h_q + rg - 1) / rg;
+  p.causal = 0;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.kv = kv;
+  p.indices = indices;
+  p.topk = topk;
+  p.vq = s_q;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int e = mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
+  if (e != 0) return MLA_ERR_CUDA;
+  mla::CombineParams cp{};
+  cp.num_splits = num_splits;
+  cp.o_part = p.o_part;
+  cp.lse_part = p.lse_part;
+  cp.out = p.out;
+  cp.lse = lse;
+  cp.batch = s_q;
+  cp.s_q = s_q;
+  cp.h_q = h_q;
+  cp.rows = h_q;
+  cp.vq = s_q;
+  e = mla::launch_combine(cp, st);
+  return e == 0 ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int mla_read_status(void* workspace, int reset, int* status, void* stream) {
   if (!workspace || !status) return MLA_ERR_NULL_POINTER;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -336,8 +336,9 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
     int b, c0, c1, split;
     while (ok && walk.next(p, b, c0, c1, split)) {
       const int breal = b / p.vq;
-      const int L = p.cache_seqlens[breal];
-      const int32_t* bt = p.block_table + static_cast<long long>(breal) * p.max_blocks;
+      // sparse prefill: one contiguous cache of kv_len tokens (no length array, no block table)
+      const int L = p.cache_seqlens ? p.cache_seqlens[breal] : p.kv_len;
+      const int32_t* bt = p.block_table ? p.block_table + static_cast<long long>(breal) * p.max_blocks : nullptr;
       const int32_t* ind = p.indices + static_cast<long long>(b) * p.topk;
       if (lane == 0) {
         ok = mbar_wait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc);
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
           const int r = lane + 32 * k;
           const int pos = (c0 + t) * kBlockTokens + r;
           const int idx = pos < p.topk ? ind[pos] : -1;
-          row_tab[r] = (idx >= 0 && idx < L) ? bt[idx >> 6] * kPage + (idx & (kPage - 1)) : -1;
+          row_tab[r] = (idx >= 0 && idx < L) ? (bt ? bt[idx >> 6] * kPage + (idx & (kPage - 1)) : idx) : -1;
         }
         __syncwarp();
       };
@@ -593,7 +594,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
     ChunkWalk walk(p, part);
     int b, c0, c1, split;
     while (walk.next(p, b, c0, c1, split)) {
-      const int L = p.cache_seqlens[SPARSE ? b / p.vq : b];
+      const int L = !SPARSE ? p.cache_seqlens[b] : (p.cache_seqlens ? p.cache_seqlens[b / p.vq] : p.kv_len);
       const int n = c1 - c0;
       const bool single = (p.num_splits[b + 1] - p.num_splits[b]) == 1;
       const int row0 = rg * RG;

@@ -46,6 +46,7 @@ struct DecodeParams {
   const int32_t* indices; // [batch * s_q, topk] logical cache positions; others: empty slots
   int topk;
   int vq;
+  int kv_len;             // sparse prefill: tokens of the one contiguous cache (cache_seqlens null)
 };
 
 struct CombineParams {

@@ -122,6 +122,27 @@ def oracle_baseline(case, budget_s: float = 15.0):
     import mla_inputs as mi
     t0 = time.perf_counter()
     done = []
+    if case.meta.get("prefill"):
+        # sparse prefill: the oracle over the first query tokens, as many as the budget allows
+        s_kv = int(case.cache_seqlens[0])
+        kv_rows = case.kv.reshape(-1, case.kv.shape[-1])[:s_kv]
+        n = 0
+        while n < case.s_q:
+            oracle.mla_sparse_prefill_reference(case.q_bits[0, n:n + 1], kv_rows, case.indices[0, n:n + 1],
+                                                case.softmax_scale)
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        sub = mi.DecodeCase(**{**case.__dict__, "q_bits": case.q_bits[:, :n], "s_q": n,
+                               "indices": case.indices[:, :n]})
+        try:
+            from threadpoolctl import threadpool_info
+            cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        except Exception:
+            cores = os.cpu_count() or 1
+        return {"seconds": dt, "requests": n, "units": mi.workload_units(sub), "cores": int(cores),
+                "what": f"first {n} of {case.s_q} query tokens"}
     for b in range(case.batch):
         if case.indices is not None:
             oracle.mla_sparse_decode_reference(case, case.indices, requests=[b])
@@ -140,7 +161,8 @@ def oracle_baseline(case, budget_s: float = 15.0):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         cores = os.cpu_count() or 1
-    return {"seconds": dt, "requests": len(done), "units": units, "cores": int(cores)}
+    return {"seconds": dt, "requests": len(done), "units": units, "cores": int(cores),
+            "what": f"first {len(done)} of {case.batch} requests"}
 
 
 # DRAM bytes (read + write) per launch of the main kernel from an ncu capture of the current
@@ -155,7 +177,11 @@ def rank_case(workload: str, rank: int, batch=None):
     import mla_inputs as mi
     w = mi.WORKLOADS[workload]
     case = mi.make_workload(workload, poison=False, batch=batch)
-    if rank > 0:
+    if rank > 0 and w.prefill:
+        s_kv = int(case.cache_seqlens[0])
+        case = mi.make_prefill_case(w.s_q, w.h_q, s_kv, w.topk, w.seed + 1000 * rank, name=workload)
+        case.meta["prefill"] = True
+    elif rank > 0:
         idx = case.indices
         case = mi.make_case(case.batch, case.s_q, case.h_q, case.cache_seqlens, causal=case.causal,
                             kv_format=case.kv_format, seed=w.seed + 1000 * rank, poison=False, name=workload)
@@ -219,7 +245,7 @@ def main():
                                                  "h_q": w.h_q, "seqlens": w.seqlens, "kv": w.kv_format,
                                                  "topk": w.topk},
                 "cpu_baseline": {"value": value, "unit": "GB/s", "cores": timed[0]["cores"], "kind": "oracle",
-                                 "sample": f"first {timed[0]['requests']} of {w.batch} requests per step"},
+                                 "sample": timed[0]["what"] + " per step"},
                 "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -256,6 +282,15 @@ def main():
     lse = torch.empty((case.batch, case.h_q, case.s_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    prefill = bool(case.meta.get("prefill"))
+    if prefill:
+        s_kv = int(case.cache_seqlens[0])
+        kv = kv.reshape(-1, mi.D_QK)[:s_kv].reshape(s_kv, 1, mi.D_QK).contiguous()
+        q = q[0].contiguous()
+        idx = idx[0].contiguous()
+        out = out[0]
+        lse = lse[0]
+
     def metadata(sl_):
         if sparse:
             return mla.mla_get_metadata_sparse(case.batch, case.s_q, case.topk, case.h_q, 1, num_sm_parts=parts,
@@ -263,7 +298,10 @@ def main():
         return mla.mla_get_metadata(sl_, R, 1, num_sm_parts=parts)
 
     def decode(q_, bt_, sl_, idx_, md, ns):
-        if sparse:
+        if prefill:
+            mla.mla_sparse_prefill(q_, kv, idx_, case.softmax_scale, tile_md=md, num_splits=ns, out=out, lse=lse,
+                                   workspace=ws)
+        elif sparse:
             mla.mla_decode_kvcache_sparse(q_, kv, bt_, sl_, idx_, 512, md, ns, softmax_scale=case.softmax_scale,
                                           out=out, lse=lse, workspace=ws)
         else:
@@ -383,7 +421,7 @@ def main():
         r = oracle_baseline(case, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": r["units"]["bytes"] / r["seconds"] / 1e9, "unit": "GB/s",
                                 "cores": r["cores"], "kind": "oracle",
-                                "sample": f"first {r['requests']} of {case.batch} requests, fp64 numpy"}
+                                "sample": r["what"] + ", fp64 numpy"}
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -180,6 +180,21 @@ MLA_API int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_
                                       float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Sparse prefill (flash_mla_sparse_fwd(q, kv, indices, sm_scale, d_v = 512) on the gitcode
+ * FlashMLA page, "稀疏预填充使用"): every query token attends to the listed tokens of one
+ * contiguous cache, with the reading of the token-sparse decode above.
+ *   q        device bf16 [s_q, h_q, 576];   kv  device bf16 [s_kv, 1, 576] (16-byte aligned)
+ *   indices  device int32 [s_q, 1, topk]: positions in [0, s_kv), others are empty slots
+ *   tile_md, num_splits   from mla_get_metadata_sparse(1, s_q, topk, h_q, h_kv, ...)
+ *   out      device bf16 [s_q, h_q, 512];  lse  device fp32 [h_q, s_q] (natural log)
+ *   workspace  >= mla_workspace_size(s_q, num_sm_parts, h_q, h_kv) bytes
+ */
+MLA_API int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const int32_t* indices, int s_q, int h_q,
+                               int h_kv, int d_v, int topk, const int32_t* tile_md, int num_sm_parts,
+                               const int32_t* num_splits, float softmax_scale, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Reads the device status word of a workspace into *status (host pointer).  This call
  * synchronises `stream`.  reset != 0 clears the word afterwards (enqueued on `stream`).
  */

@@ -102,6 +102,7 @@ class Workload:
     seed: int
     description: str
     topk: int = 0                 # > 0: token-sparse decode over topk cache positions per query
+    prefill: bool = False         # sparse prefill: batch 1, s_q query tokens, one contiguous cache
 
 
 WORKLOADS = {
@@ -124,6 +125,10 @@ WORKLOADS = {
         "sparse_b128_h128_L8192_topk2048", 128, 1, 128, "fixed:8192", False, "bf16", 6,
         "token-sparse decode: batch 128, s_q 1, h_q 128, every cache_seqlen 8192, 2048 distinct "
         "cache positions per query in random order", topk=2048),
+    "sparse_prefill_s4096_h128_kv8192_topk2048": Workload(
+        "sparse_prefill_s4096_h128_kv8192_topk2048", 1, 4096, 128, "fixed:8192", False, "bf16", 7,
+        "sparse prefill: 4096 query tokens of 128 heads over one contiguous 8192-token cache, 2048 "
+        "distinct listed positions per query token in random order", topk=2048, prefill=True),
 }
 
 
@@ -322,11 +327,34 @@ def make_sparse_indices(cache_seqlens, s_q: int, topk: int, seed: int, *, invali
     return out
 
 
+def make_prefill_case(s_q: int, h_q: int, s_kv: int, topk: int, seed: int, *, invalid_frac: float = 0.0,
+                      softmax_scale: Optional[float] = None, name: str = "") -> DecodeCase:
+    """Sparse prefill inputs as a one-request case: s_q query tokens of h_q heads, one
+    contiguous cache of s_kv tokens (pages in order: block_table = 0, 1, 2, ...; the prefill
+    call reads kv = the first s_kv rows of case.kv), indices int32 [1, s_q, topk]."""
+    n_pages = (int(s_kv) + PAGE - 1) // PAGE
+    q = f32_to_bf16_bits(_normal_f32(seed, _S_Q, s_q * h_q * D_QK)).reshape(1, s_q, h_q, D_QK)
+    kv = _gen_kv(seed, n_pages, "bf16")
+    bt = np.arange(n_pages, dtype=np.int32).reshape(1, n_pages)
+    sl = np.asarray([s_kv], dtype=np.int32)
+    case = DecodeCase(q_bits=q, kv=kv, block_table=bt, cache_seqlens=sl, s_q=s_q, h_q=h_q, causal=False,
+                      softmax_scale=float(softmax_scale if softmax_scale is not None else D_QK ** -0.5),
+                      kv_format="bf16", name=name)
+    case.indices = make_sparse_indices(sl, s_q, topk, seed, invalid_frac=invalid_frac)
+    return case
+
+
 def make_workload(name: str, *, batch: Optional[int] = None, poison: bool = True,
                   spare_blocks: int = 0) -> DecodeCase:
     """One of the named decode workloads at its full size (or with ``batch`` requests:
     the first ``batch`` of the full draw of cache lengths)."""
     w = WORKLOADS[name]
+    if w.prefill:
+        s_kv = int(w.seqlens.partition(":")[2])
+        case = make_prefill_case(w.s_q, w.h_q, s_kv, w.topk, w.seed, name=name)
+        case.meta["workload"] = w.description
+        case.meta["prefill"] = True
+        return case
     seqlens = draw_seqlens(w.seqlens, w.batch, w.seed)
     b = w.batch if batch is None else int(batch)
     if b != w.batch:
@@ -345,10 +373,12 @@ def workload_units(case: DecodeCase) -> dict:
     L = case.cache_seqlens.astype(np.int64)
     R = case.rows
     if case.indices is not None:
-        # token-sparse: each query position reads and attends to its valid listed positions
+        # token-sparse: each query position attends to its valid listed positions; the cache
+        # bytes are those of the distinct positions each request lists (read once at best)
         valid = (case.indices >= 0) & (case.indices < L[:, None, None])
         n_sel = int(valid.sum())
-        kv_bytes = n_sel * case.kv_bytes_per_token()
+        distinct = sum(int(np.unique(case.indices[b][valid[b]]).size) for b in range(case.batch))
+        kv_bytes = distinct * case.kv_bytes_per_token()
         qob = case.batch * R * (D_QK * 2 + D_V * 2 + 4) + case.indices.size * 4
         pairs = n_sel * case.h_q
         return {"kv_bytes": kv_bytes, "kv_bytes_paged": kv_bytes, "bytes": kv_bytes + qob,
@@ -374,5 +404,5 @@ __all__ = [
     "D_QK", "D_V", "D_ROPE", "PAGE", "FP8_TOKEN_BYTES", "FP8_GROUP", "E4M3_MAX",
     "DecodeCase", "Workload", "WORKLOADS", "make_case", "make_workload", "make_block_table",
     "draw_seqlens", "poison_unused", "f32_to_bf16_bits", "bf16_bits_to_f32", "workload_units",
-    "make_sparse_indices",
+    "make_sparse_indices", "make_prefill_case",
 ]

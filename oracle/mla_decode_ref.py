@@ -137,3 +137,30 @@ def mla_sparse_decode_reference(case, indices, requests=None):
             O[b, i] = o
             LSE[b, :, i] = l
     return O, LSE
+
+
+def mla_sparse_prefill_reference(q_bits, kv_bits, indices, softmax_scale: float):
+    """Sparse prefill (flash_mla_sparse_fwd(q, kv, indices, sm_scale, d_v = 512) on the gitcode
+    FlashMLA page, "稀疏预填充使用"), by definition, in fp64: query token i, head h attends to
+    the rows kv[indices[i, k]] with 0 <= indices[i, k] < s_kv (other entries are empty slots):
+
+      s_k = softmax_scale * q[i, h] . kv[indices[i, k]],  LSE = log sum_k exp(s_k),
+      O   = sum_k exp(s_k - LSE) * kv[indices[i, k]][:512]
+
+    q_bits bf16 bits [s_q, h_q, 576], kv_bits bf16 bits [s_kv, 576], indices [s_q, topk].
+    Returns (O fp64 [s_q, h_q, 512], LSE fp64 [h_q, s_q]); no valid entry: O = 0, LSE = -inf.
+    """
+    q = bf16_to_f64(q_bits)
+    kv = bf16_to_f64(kv_bits)
+    s_kv = kv.shape[0]
+    s_q, h_q = q.shape[0], q.shape[1]
+    O = np.zeros((s_q, h_q, D_V), dtype=np.float64)
+    LSE = np.full((h_q, s_q), -np.inf, dtype=np.float64)
+    for i in range(s_q):
+        sel = [int(j) for j in np.asarray(indices[i]).reshape(-1) if 0 <= int(j) < s_kv]
+        if not sel:
+            continue
+        o, l = attend_rows(q[i], kv[sel], np.full(h_q, len(sel)), softmax_scale)
+        O[i] = o
+        LSE[:, i] = l
+    return O, LSE

@@ -39,6 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
     names = _declared()
     assert set(names) == {"mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
                           "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
+                          "mla_sparse_prefill",
                           "mla_read_status", "mla_strerror", "mla_version"}
     so = os.path.join(ROOT, "attention_mla_get_b200", "libmla.so")
     nm = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True).stdout

@@ -105,3 +105,53 @@ def test_full_sparse_workload_sampled():
     sample = [0, 57, case.batch - 1]
     O_ref, L_ref = oracle.mla_sparse_decode_reference(case, case.indices, requests=sample)
     compare(case, out, lse, O_ref, L_ref, requests=sample)
+
+
+# ---------------------------------------------------------------- sparse prefill
+PREFILL_CASES = [
+    # (name, s_q, h_q, s_kv, topk, invalid_frac)
+    ("pf_r16", 37, 16, 1000, 128, 0.1),
+    ("pf_r64_ragged_kv", 64, 64, 777, 256, 0.0),
+    ("pf_r128", 16, 128, 4096, 512, 0.05),
+    ("pf_r32_many_tokens", 200, 32, 300, 64, 0.2),
+]
+
+
+def run_prefill(case, num_sm_parts=None):
+    import attention_mla_get_b200 as mla
+    s_kv = int(case.cache_seqlens[0])
+    q = torch.from_numpy(case.q_bits[0].view(np.int16)).view(torch.bfloat16).cuda()
+    kv = torch.from_numpy(np.ascontiguousarray(case.kv.reshape(-1, mi.D_QK)[:s_kv]).view(np.int16)).view(
+        torch.bfloat16).reshape(s_kv, 1, mi.D_QK).cuda()
+    idx = torch.from_numpy(np.ascontiguousarray(case.indices[0])).cuda()
+    md, ns = mla.mla_get_metadata_sparse(1, case.s_q, idx.shape[-1], case.h_q, 1, num_sm_parts=num_sm_parts)
+    ws = torch.zeros(mla.mla_workspace_size(case.s_q, md.shape[0], case.h_q, 1), dtype=torch.uint8, device="cuda")
+    out, lse = mla.mla_sparse_prefill(q, kv, idx, case.softmax_scale, tile_md=md, num_splits=ns, workspace=ws)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), lse.cpu().numpy(), mla.mla_read_status(ws)
+
+
+@pytest.mark.parametrize("name,s_q,h_q,s_kv,topk,inv", PREFILL_CASES, ids=[c[0] for c in PREFILL_CASES])
+@pytest.mark.parametrize("parts", [None, 5])
+def test_sparse_prefill_parity(name, s_q, h_q, s_kv, topk, inv, parts):
+    case = mi.make_prefill_case(s_q, h_q, s_kv, topk, seed=zlib.crc32(name.encode()) % 1000, invalid_frac=inv)
+    s_kv_rows = case.kv.reshape(-1, mi.D_QK)[:s_kv]
+    O_ref, L_ref = oracle.mla_sparse_prefill_reference(case.q_bits[0], s_kv_rows, case.indices[0],
+                                                       case.softmax_scale)
+    out, lse, status = run_prefill(case, num_sm_parts=parts)
+    assert status == 0
+    compare(case, out[None], lse[None], O_ref[None], L_ref[None])
+
+
+def test_flash_mla_sparse_fwd_spelling():
+    import attention_mla_get_b200 as mla
+    case = mi.make_prefill_case(8, 16, 500, 64, seed=77)
+    q = torch.from_numpy(case.q_bits[0].view(np.int16)).view(torch.bfloat16).cuda()
+    kv = torch.from_numpy(np.ascontiguousarray(case.kv.reshape(-1, mi.D_QK)[:500]).view(np.int16)).view(
+        torch.bfloat16).reshape(500, 1, mi.D_QK).cuda()
+    idx = torch.from_numpy(np.ascontiguousarray(case.indices[0])).reshape(8, 1, 64).cuda()
+    out, lse = mla.flash_mla_sparse_fwd(q, kv, idx, case.softmax_scale, d_v=512)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle.mla_sparse_prefill_reference(case.q_bits[0], case.kv.reshape(-1, mi.D_QK)[:500],
+                                                       case.indices[0], case.softmax_scale)
+    compare(case, out.float().cpu().numpy()[None], lse.cpu().numpy()[None], O_ref[None], L_ref[None])

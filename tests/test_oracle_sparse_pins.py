@@ -183,3 +183,38 @@ def test_planted_value_offset(monkeypatch):
     monkeypatch.setattr(ref, "gather_request_keys", bad)
     assert check_brute_force() > 1e-6
     assert check_single_entry() > 1e-6
+
+
+# --------------------------------------------------------------- sparse prefill
+def _prefill_kv(case):
+    s_kv = int(case.cache_seqlens[0])
+    return case.kv.reshape(-1, case.kv.shape[-1])[:s_kv]
+
+
+def check_prefill_brute_force():
+    case = mi.make_prefill_case(3, 2, 150, 20, seed=31, invalid_frac=0.2)
+    O, L = oracle.mla_sparse_prefill_reference(case.q_bits[0], _prefill_kv(case), case.indices[0], case.softmax_scale)
+    Ob, Lb = brute_force_sparse(case, case.indices)          # one request, identity block table
+    return _err(O - Ob[0], L - Lb[0])
+
+
+def test_prefill_brute_force():
+    assert check_prefill_brute_force() < 1e-11
+
+
+def test_prefill_is_one_request_of_sparse_decode():
+    case = mi.make_prefill_case(5, 3, 333, 64, seed=32, invalid_frac=0.1)
+    O, L = oracle.mla_sparse_prefill_reference(case.q_bits[0], _prefill_kv(case), case.indices[0], case.softmax_scale)
+    Od, Ld = oracle.mla_sparse_decode_reference(case, case.indices)
+    assert _err(O - Od[0], L - Ld[0]) < 1e-12
+
+
+def test_planted_prefill_row_offset(monkeypatch):
+    real = ref.attend_rows
+
+    def bad(qrows, K, n_visible, scale):
+        K2 = K.copy()
+        K2[:, :512] = np.roll(K[:, :512], 1, axis=0)                  # values of the wrong rows
+        return real(qrows, K2, n_visible, scale)
+    monkeypatch.setattr(ref, "attend_rows", bad)
+    assert check_prefill_brute_force() > 1e-6
