@@ -78,7 +78,7 @@ struct Cfg {
   static constexpr int kOffRaw = kOffSlots + kNumSlots * kSlotBytes;
   static constexpr int kOffScale = kOffRaw + kNumRaw * kRawBytes;
   static constexpr int kOffMisc = kOffScale + kNumScale * kScaleBytes;
-  static constexpr int kMiscBytes = 3584;  // + 512 B: token-sparse row table
+  static constexpr int kMiscBytes = FP8 ? 3072 : 6656;  // bf16: + 7 x 512 B of token-sparse row tables
   static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
   static constexpr uint32_t kPSwzMask = RG / 8 - 1;                // (row bytes / 16) - 1
   static constexpr uint32_t kPLayout = RG == 64 ? kSwizzle128 : (RG == 32 ? kSwizzle64 : kSwizzle32);
@@ -242,8 +242,13 @@ __device__ __forceinline__ StepPages step_pages(const int32_t* bt, int st, int n
 // SPARSE (bf16 cache only): token-sparse decode.  A "request" b of the chunk walk is the query
 // position (b / vq, b % vq) with topk listed cache positions; the producer warp copies the
 // listed tokens' rows (16-byte cp.async per lane, zeros for empty slots) instead of TMA pages.
+// token-sparse: warps 4 and 6-11 gather (warp 4 also loads Q)
+constexpr int kGatherWarps = 7;
+template <int RG, bool FP8, bool SPARSE>
+constexpr int threads_of() { return SPARSE ? 384 : Cfg<RG, FP8>::kThreads; }
+
 template <int RG, bool FP8, bool SPARSE = false>
-__global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
+__global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                       const __grid_constant__ CUtensorMap tm_scale, const __grid_constant__ CUtensorMap tm_rope,
                       const DecodeParams p) {
@@ -264,7 +269,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
   float* m_sm = reinterpret_cast<float*>(misc + 2048);      // [64]
   float* alpha_sm = reinterpret_cast<float*>(misc + 2304);  // [64]
   float* inv_sm = reinterpret_cast<float*>(misc + 2560);    // [64]
-  int32_t* row_tab = reinterpret_cast<int32_t*>(misc + 3072);  // [128] SPARSE: cache row per token slot
+  int32_t* row_tabs = reinterpret_cast<int32_t*>(misc + 3072);  // SPARSE [7][128]: cache row per token slot
   static_assert(kNumBars * 8 <= 512, "barrier area");
   auto bar = [&](int i) -> uint32_t { return sBars + 8u * static_cast<uint32_t>(i); };
 
@@ -276,7 +281,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMaxSlots; ++i) {
-      mbar_init(bar(kBarSlotFull + i), SPARSE ? 32 : 1);  // SPARSE: one cp.async arrival per lane
+      mbar_init(bar(kBarSlotFull + i), SPARSE ? 32 * kGatherWarps : 1);  // SPARSE: a cp.async arrival per lane
       mbar_init(bar(kBarSlotEmpty + i), 1);
     }
     for (int i = 0; i < kNumS; ++i) {
@@ -322,12 +327,16 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
 
   pdl_launch_dependents();
 
-  if (SPARSE && warp == 4) {
-    // ======================== gather producer (token-sparse) =======================
-    // The 128 listed tokens of a step are looked up once per step group (row_tab: physical cache
-    // row, -1 for an empty slot); then every warp-wide cp.async copies whole 16-byte chunks of
-    // two (or four) token rows, so each instruction reads a few contiguous row segments.  The
-    // slot's full barrier counts one arrival per lane, made when that lane's copies landed.
+  if (SPARSE && (warp == 4 || warp >= 6)) {
+    // ======================= gather producers (token-sparse) =======================
+    // Seven warps fill every slot together (more copies in flight).  Each looks up the 128 listed
+    // tokens of a step once per step group into its own row table (physical cache row, -1 for
+    // an empty slot); every warp-wide cp.async then copies 16-byte chunks of two (or four) token
+    // rows, so each instruction reads a few contiguous row segments, and warp gw issues every
+    // seventh of them.  The slot's full barrier counts one arrival per lane of the seven warps,
+    // made when that lane's copies landed.
+    const int gw = warp == 4 ? 0 : warp - 5;
+    int32_t* row_tab = row_tabs + 128 * gw;
     uint32_t g = 0;
     int q_fills = 0;
     bool ok = true;
@@ -340,16 +349,19 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
       const int L = p.cache_seqlens ? p.cache_seqlens[breal] : p.kv_len;
       const int32_t* bt = p.block_table ? p.block_table + static_cast<long long>(breal) * p.max_blocks : nullptr;
       const int32_t* ind = p.indices + static_cast<long long>(b) * p.topk;
-      if (lane == 0) {
-        ok = mbar_wait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc);
-        if (ok) {
-          mbar_arrive_expect_tx(bar(kBarQFull), 9u * C::kQAtomBytes);
-          for (int a = 0; a < 9; ++a) tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, 64 * a, rg * RG, b, bar(kBarQFull));
+      if (gw == 0) {
+        if (lane == 0) {
+          ok = mbar_wait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc);
+          if (ok) {
+            mbar_arrive_expect_tx(bar(kBarQFull), 9u * C::kQAtomBytes);
+            for (int a = 0; a < 9; ++a)
+              tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, 64 * a, rg * RG, b, bar(kBarQFull));
+          }
         }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        ++q_fills;
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      ++q_fills;
       const int n = c1 - c0;
       auto rows_of = [&](int t) {
         __syncwarp();  // the previous group's copies were all issued
@@ -373,7 +385,7 @@ __global__ void __launch_bounds__(Cfg<RG, FP8>::kThreads, 1)
         const int sub = lane / cpr, c = lane % cpr;
         const uint32_t a = static_cast<uint32_t>(c >> 3), cc = static_cast<uint32_t>(c & 7);
         const char* src0 = kvb + (dims0 + 8 * c) * 2;
-        for (int i = 0; i < kBlockTokens / rpi; ++i) {
+        for (int i = gw; i < kBlockTokens / rpi; i += kGatherWarps) {
           const uint32_t r = static_cast<uint32_t>(i * rpi + sub);
           const int row = row_tab[r];
           cp_async_16(dst + a * C::kAtomColBytes + r * 128u + ((cc ^ (r & 7u)) << 4),
@@ -896,10 +908,11 @@ int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtenso
                 const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
   using C = Cfg<RG, FP8>;
   auto kern = mla_decode_kernel<RG, FP8, SPARSE>;
+  constexpr int kThreads = threads_of<RG, FP8, SPARSE>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid(p.num_sm_parts, p.row_groups, 1);
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, tm_scale, tm_rope, p);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, tm_scale, tm_rope, p);
   return static_cast<int>(cudaGetLastError());
 }
 
