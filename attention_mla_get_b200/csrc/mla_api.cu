@@ -252,7 +252,8 @@ int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_t num_bl
 
   EncodeTiledFn encode = encode_fn();
   if (!encode) return MLA_ERR_CUDA;
-  const int rg = rows_per_cta_for(h_q);
+  const bool pair = mla::use_pair_kernel(h_q, false);  // more than 64 heads: CTA pairs of 128
+  const int rg = pair ? mla::kRowsPerCta : rows_per_cta_for(h_q);
   // q as {576 dims, h_q heads, batch * s_q positions}; one box = 64 dims x rg heads of a position
   CUtensorMap tm_q;
   {
@@ -283,7 +284,7 @@ int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_t num_bl
   p.s_q = s_q;
   p.h_q = h_q;
   p.rows = h_q;
-  p.row_groups = (h_q + rg - 1) / rg;
+  p.row_groups = pair ? (h_q + mla::kPairRows - 1) / mla::kPairRows : (h_q + rg - 1) / rg;
   p.causal = 0;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.kv = kvcache;
@@ -291,7 +292,7 @@ int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_t num_bl
   p.topk = topk;
   p.vq = s_q;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
+  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, p, st) : mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
   mla::CombineParams cp{};
   cp.num_splits = num_splits;
@@ -325,7 +326,8 @@ int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const int32_t* i
   if (workspace_bytes < wl.total) return MLA_ERR_WORKSPACE;
   EncodeTiledFn encode = encode_fn();
   if (!encode) return MLA_ERR_CUDA;
-  const int rg = rows_per_cta_for(h_q);
+  const bool pair = mla::use_pair_kernel(h_q, false);  // more than 64 heads: CTA pairs of 128
+  const int rg = pair ? mla::kRowsPerCta : rows_per_cta_for(h_q);
   CUtensorMap tm_q;  // {576 dims, h_q heads, s_q query tokens}
   {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(h_q), static_cast<cuuint64_t>(s_q)};
@@ -354,7 +356,7 @@ int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const int32_t* i
   p.s_q = s_q;
   p.h_q = h_q;
   p.rows = h_q;
-  p.row_groups = (h_q + rg - 1) / rg;
+  p.row_groups = pair ? (h_q + mla::kPairRows - 1) / mla::kPairRows : (h_q + rg - 1) / rg;
   p.causal = 0;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.kv = kv;
@@ -362,7 +364,7 @@ int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const int32_t* i
   p.topk = topk;
   p.vq = s_q;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
+  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, p, st) : mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
   mla::CombineParams cp{};
   cp.num_splits = num_splits;

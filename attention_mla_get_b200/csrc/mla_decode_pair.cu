@@ -91,16 +91,18 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, 
   return idesc_bf16(M, N, a_mn_major, b_mn_major) & ~((7u << 7) | (7u << 10));
 }
 
-template <bool FP8>
+template <bool FP8, bool SPARSE = false>
 struct PairCfg {
-  // FP8: 16 warps (two idle) so that the compiler keeps every thread within 128 registers, the
-  // per-SM-sub-partition share of 4 resident warps
-  static constexpr int kThreads = FP8 ? 512 : 320;
+  // FP8 and token-sparse: 16 warps (FP8: two idle) so that the compiler keeps every thread
+  // within 128 registers, the per-SM-sub-partition share of 4 resident warps
+  static constexpr int kThreads = (FP8 || SPARSE) ? 512 : 320;
   static constexpr int kNumSlots = FP8 ? 2 : 3;  // FP8 gives a stage to the raw ring
   static constexpr int kOffRaw = kOffSlots + kNumSlots * kSlotBytes;
   static constexpr int kOffRope = kOffRaw + (FP8 ? kNumRaw * kRawBytes : 0);
   static constexpr int kOffMisc = kOffRope + kRopeBytes;
-  static constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+  // token-sparse: + 1 KB for the row table of a step's 256 listed tokens
+  static constexpr int kMisc = kMiscBytes + (SPARSE ? 1024 : 0);
+  static constexpr int kSmemBytes = kOffMisc + kMisc + 1024;  // + alignment slack
   static constexpr uint32_t kIdescQK = FP8 ? idesc_f16(256, kRows, false, false) : idesc_bf16(256, kRows, false, false);
   static constexpr uint32_t kIdescPV = FP8 ? idesc_f16(256, kRows, true, true) : idesc_bf16(256, kRows, true, true);
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -136,7 +138,10 @@ enum : int {
   kBarRawEmpty = kBarRawFull + kNumRaw,       // [2] FP8, both: this CTA's dequant warps
   kBarQReady = kBarRawEmpty + kNumRaw,        // FP8, leader: Q in f16 (every dequant warp, both CTAs)
   kBarRopeReady = kBarQReady + 1,             // FP8, leader: RoPE slot in f16 (as kBarQReady)
-  kNumBars = kBarRopeReady + 1,
+  // token-sparse, both: this CTA's gather warps' cp.async landed ([stages], then RoPE slot)
+  kBarGather = kBarRopeReady + 1,
+  kBarGatherRope = kBarGather + kMaxSlots,
+  kNumBars = kBarGatherRope + 1,
 };
 constexpr int kMiscHolder = 512;   // TMEM base address
 constexpr int kMiscAbort = 516;    // abort flag
@@ -149,6 +154,8 @@ constexpr int kMiscAlpha = 3584;   // float [128]
 constexpr int kMiscInv = 4096;     // float [128]
 constexpr int kMiscXMax = 4608;    // float [2][128]: the peer's block maxima
 constexpr int kMiscXL = 5632;      // float [128]: the peer's row sums
+constexpr int kMiscRowTab = 6144;  // token-sparse: int32 [256] cache rows of a step's listed tokens
+constexpr int kGatherThreads = 192;  // token-sparse: warps 10-15 copy the listed tokens' rows
 static_assert(kNumBars * 8 <= kMiscHolder, "barrier area");
 static_assert(kMiscXL + 512 <= kMiscBytes, "misc area");
 
@@ -166,7 +173,8 @@ struct ChunkWalk {
   }
   __device__ bool next(const DecodeParams& p, int& cb, int& c0, int& c1, int& csplit) {
     while (b < end_b || (b == end_b && blk < end_blk)) {
-      const int n = blocks_of(p.cache_seqlens[b]);
+      // token-sparse: every query position is a request of topk listed positions
+      const int n = blocks_of(p.topk > 0 ? p.topk : p.cache_seqlens[b]);
       const int stop = (b == end_b) ? end_blk : n;
       cb = b;
       c0 = blk;
@@ -329,12 +337,15 @@ __device__ __forceinline__ void dequant_row(uint32_t src, uint32_t dst, uint32_t
   }
 }
 
-template <bool FP8>
-__global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
+// SPARSE (bf16 cache): token-sparse decode, every query position a request of topk listed
+// cache positions (see mla_decode.cu); warps 10-15 copy the listed tokens' rows into the stages
+// with 16-byte cp.async and the producer thread forwards each stage's completion to the leader.
+template <bool FP8, bool SPARSE = false>
+__global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                            const __grid_constant__ CUtensorMap tm_scale, const __grid_constant__ CUtensorMap tm_rope,
                            const DecodeParams p) {
-  using C = PairCfg<FP8>;
+  using C = PairCfg<FP8, SPARSE>;
   constexpr int kNumSlots = C::kNumSlots;
   constexpr uint32_t kIdescQK = C::kIdescQK;
   constexpr uint32_t kIdescPV = C::kIdescPV;
@@ -399,6 +410,8 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
     }
     mbar_init(bar(kBarQReady), 2 * kDequantThreads / 32);
     mbar_init(bar(kBarRopeReady), 2 * kDequantThreads / 32);
+    for (int i = 0; i < kMaxSlots; ++i) mbar_init(bar(kBarGather + i), kGatherThreads);  // cp.async arrivals
+    mbar_init(bar(kBarGatherRope), kGatherThreads);
     *abort_flag = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerFills) = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerQ) = 0;
@@ -498,9 +511,9 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
         return true;
       };
       while (ok && walk.next(p, b, c0, c1, split)) {
-        const int L = p.cache_seqlens[b];
+        const int L = SPARSE ? 0 : p.cache_seqlens[b];  // token-sparse: b is a query position
         const int npages = (L + kPage - 1) / kPage;
-        const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
+        const int32_t* bt = SPARSE ? nullptr : p.block_table + static_cast<long long>(b) * p.max_blocks;
         if (!pwait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc)) break;
         if (FP8) {
           // this CTA's copy; its dequant warps convert Q to f16 before the leader's MMA uses it
@@ -517,7 +530,34 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
         }
         ++q_fills;
         const int n = (c1 - c0 + 1) / 2;
-        for (int e = 0; ok && e < 2 * n; ++e) {
+        if (SPARSE) {
+          // token-sparse: this CTA's gather warps fill the stages; pass each one's completion on
+          // to the leader's full barrier, in the fill order (their copies are generic-proxy
+          // writes, hence the proxy fence before the arrive)
+          auto forward = [&]() -> bool {
+            const int s = static_cast<int>(fills % kNumSlots);
+            const uint32_t use = fills / kNumSlots;
+            if (!pwait(bar(kBarGather + s), use & 1u, wc)) return false;
+            fence_proxy_async_smem();
+            mbar_arrive_remote(lead(bar(kBarSlotFull + s)));
+            last_use[s] = static_cast<int>(use);
+            ++fills;
+            return true;
+          };
+          for (int e = 0; ok && e < 2 * n; ++e) {
+            bool is_v;
+            int t;
+            order_at(e, n, is_v, t);
+            if (!is_v) {
+              if (!pwait(bar(kBarGatherRope), static_cast<uint32_t>(rope_fills) & 1u, wc)) { ok = false; break; }
+              fence_proxy_async_smem();
+              mbar_arrive_remote(lead(bar(kBarRopeFull)));
+              ++rope_fills;
+            }
+            for (int k = 0; ok && k < 4; ++k) ok = forward();
+          }
+        }
+        for (int e = 0; ok && !SPARSE && e < 2 * n; ++e) {
           bool is_v;
           int t;
           order_at(e, n, is_v, t);
@@ -637,7 +677,7 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
       const uint64_t kdesc0 = smem_desc(sSlots, 16, 1024, kSwizzle128);
       const uint64_t vdesc0 = smem_desc(sSlots, kBoxBytes, 1024, kSwizzle128);
       while (ok && walk.next(p, b, c0, c1, split)) {
-        const int L = p.cache_seqlens[b];
+        const int L = SPARSE ? 0 : p.cache_seqlens[b];
         const int n = (c1 - c0 + 1) / 2;
         // FP8: both CTAs' dequant warps have converted their Q halves to f16
         if (!pwait(bar(FP8 ? kBarQReady : kBarQFull), chunk & 1, wc)) break;
@@ -683,7 +723,7 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
             // operands that only TMA or shared-memory stores produced
             tc_fence_after();
             // FP8 stages hold zeros for tokens outside the request (written by the dequant warps)
-            const bool tail = !FP8 && is_tail(c0, c1, t, L);
+            const bool tail = !FP8 && !SPARSE && is_tail(c0, c1, t, L);
             for (int m = 0; ok && m < 2; ++m) {
               for (int blk = 0; blk < 2; ++blk) {
                 uint32_t s;
@@ -717,6 +757,86 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
       umma_commit_pair(bar(kBarDrain));
       drain_wait(bar(kBarDrain), 0);
     }
+  } else if (SPARSE && warp >= kWarpDequant) {
+    // ======================= gather warps (token-sparse, 10-15) ======================
+    // Per step group they look up the listed tokens' cache rows once (a shared table: K(t)
+    // this CTA's 128, V(t) the step's 256), then fill the RoPE slot and the stages in the fill
+    // order with 16-byte cp.async (two or four token rows per warp instruction, every sixth
+    // instruction per warp, zeros for empty slots).  Each lane's arrival on the CTA's gather
+    // barrier completes a stage once all its copies landed; the producer thread forwards that.
+    const int gt = threadIdx.x - kWarpDequant * 32;  // 0..191
+    const int gw = gt >> 5;
+    int32_t* row_tab = reinterpret_cast<int32_t*>(misc + kMiscRowTab);
+    const char* kvb = static_cast<const char*>(p.kv);
+    uint32_t g = 0, rf = 0;
+    bool ok = true;
+    ChunkWalk walk(p, part);
+    int b, c0, c1, split;
+    bool aborted = false;
+    while (!aborted && walk.next(p, b, c0, c1, split)) {
+      const int breal = b / p.vq;
+      const int L = p.cache_seqlens ? p.cache_seqlens[breal] : p.kv_len;
+      const int32_t* bt = p.block_table ? p.block_table + static_cast<long long>(breal) * p.max_blocks : nullptr;
+      const int32_t* ind = p.indices + static_cast<long long>(b) * p.topk;
+      const int n = (c1 - c0 + 1) / 2;
+      // rows of nblk token blocks from kb0 (entry 128 q + r); false: some warp gave up (all see it)
+      auto table = [&](int kb0, int nblk) -> bool {
+        if (named_bar_any(3, kGatherThreads, !ok)) return false;  // also: the last group was issued
+        for (int e = gt; e < 128 * nblk; e += kGatherThreads) {
+          const int kb = kb0 + (e >> 7);
+          const int pos = kb * kBlockTokens + (e & 127);
+          const int idx = (kb < c1 && pos < p.topk) ? ind[pos] : -1;
+          row_tab[e] = (idx >= 0 && idx < L) ? (bt ? bt[idx >> 6] * kPage + (idx & (kPage - 1)) : idx) : -1;
+        }
+        named_bar_sync(3, kGatherThreads);
+        return true;
+      };
+      // the 128 rows of table entries tab0.. as natoms 64-dim columns from dims0: row i at
+      // dst + (i / 64) * pstride + (i % 64) * 128, column a at + a * hstride
+      auto copy = [&](uint32_t dst, int tab0, int dims0, int natoms, uint32_t pstride, uint32_t hstride) {
+        const int cpr = 8 * natoms, rpi = 32 / cpr;
+        const int sub = lane / cpr, c = lane % cpr;
+        const uint32_t a = static_cast<uint32_t>(c >> 3), cc = static_cast<uint32_t>(c & 7);
+        const char* src0 = kvb + (dims0 + 8 * c) * 2;
+        for (int it = gw; it < kBlockTokens / rpi; it += kGatherThreads / 32) {
+          const uint32_t i = static_cast<uint32_t>(it * rpi + sub);
+          const int row = row_tab[tab0 + static_cast<int>(i)];
+          cp_async_16(dst + (i >> 6) * pstride + (i & 63u) * 128u + a * hstride + ((cc ^ (i & 7u)) << 4),
+                      src0 + (row >= 0 ? static_cast<long long>(row) * (kDqk * 2) : 0), row >= 0 ? 16u : 0u);
+        }
+      };
+      auto stage = [&](int tab0, int dims0, uint32_t pstride, uint32_t hstride) -> bool {
+        const uint32_t s = g % kNumSlots, use = g / kNumSlots;
+        if (!warp_pwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc, lane)) return false;
+        copy(sSlots + s * kSlotBytes, tab0, dims0, 2, pstride, hstride);
+        cp_async_arrive_noinc(bar(kBarGather + s));
+        ++g;
+        return true;
+      };
+      for (int e = 0; e < 2 * n; ++e) {
+        bool is_v;
+        int t;
+        order_at(e, n, is_v, t);
+        if (!is_v) {
+          if (!table(c0 + 2 * t + static_cast<int>(rank), 1)) { aborted = true; break; }
+          // RoPE dims of this CTA's block ([page][64 rows][64 dims]), then K stage j: dims
+          // 128j.. as [dim half][page][64 rows][64 dims]
+          if (ok) ok = warp_pwait(bar(kBarRopeEmpty), (rf & 1u) ^ 1u, wc, lane);
+          if (ok) {
+            copy(sRope, 0, kDv, 1, kBoxBytes, 0);
+            cp_async_arrive_noinc(bar(kBarGatherRope));
+            ++rf;
+          }
+          for (int j = 0; ok && j < kKFills; ++j) ok = stage(0, 128 * j, kBoxBytes, kHalfBytes);
+        } else {
+          if (!table(c0 + 2 * t, 2)) { aborted = true; break; }
+          // V stage k = (m, blk): dims 256m + 128 rank.. of block blk as [page][dim half][64 rows]
+          for (int k = 0; ok && k < kVFills; ++k)
+            ok = stage(128 * (k & 1), 256 * (k >> 1) + 128 * static_cast<int>(rank), kHalfBytes, kBoxBytes);
+        }
+      }
+    }
+    cp_async_wait_all();  // this lane's copies have landed before the CTA may exit
   } else if (FP8 && warp >= kWarpDequant) {
     // =========================== FP8 dequant (warps 10-13) ===========================
     // Thread dt owns token row dt % 64 of page dt / 64 of each stage.  Order: per chunk the Q
@@ -842,7 +962,8 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
     ChunkWalk walk(p, part);
     int b, c0, c1, split;
     while (walk.next(p, b, c0, c1, split)) {
-      const int L = p.cache_seqlens[b];
+      // token-sparse: b is the query position (b / vq, b % vq) of a request of length L
+      const int L = !SPARSE ? p.cache_seqlens[b] : (p.cache_seqlens ? p.cache_seqlens[b / p.vq] : p.kv_len);
       const int n = (c1 - c0 + 1) / 2;
       const bool single = (p.num_splits[b + 1] - p.num_splits[b]) == 1;
       bool aborted = false;
@@ -862,11 +983,17 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
         // key j is visible to row r iff j < L, its block is in this chunk and, when causal,
         // j <= L - s_q + r / h_q, i.e. r >= (j - L + s_q) * h_q
         int cmin = -(1 << 30);
-        if (p.causal) {
-          const int i0 = j - L + p.s_q;
-          if (i0 > 0) cmin = i0 * p.h_q - row0 - 64 * h;
+        if constexpr (SPARSE) {
+          // slot j of the list is a key iff it names a position in [0, L)
+          const int idx = (kb < c1 && j < p.topk) ? p.indices[static_cast<long long>(b) * p.topk + j] : -1;
+          if (idx < 0 || idx >= L) cmin = 1 << 30;
+        } else {
+          if (p.causal) {
+            const int i0 = j - L + p.s_q;
+            if (i0 > 0) cmin = i0 * p.h_q - row0 - 64 * h;
+          }
+          if (kb >= c1 || j >= L) cmin = 1 << 30;
         }
-        if (kb >= c1 || j >= L) cmin = 1 << 30;
 #pragma unroll
         for (int c = 0; c < 64; ++c) x[c] = (c >= cmin) ? x[c] * p.scale_log2 : NEG_INF;
         // column maxima over this warp's 32 tokens; lane l keeps columns l and 32 + l
@@ -967,7 +1094,7 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
           }
           ok &= __shfl_sync(0xffffffffu, okp, 0) != 0;
         }
-        if (!FP8 && tid < kRows && is_tail(c0, c1, t, L)) {
+        if (!FP8 && !SPARSE && tid < kRows && is_tail(c0, c1, t, L)) {
           // Zero, in this CTA's V slots of the step, the rows of tokens outside the request or the
           // chunk (stale ring contents or the cache's unused page tail: 0 * NaN would poison O^T).
           // These slots count their bytes on this CTA's own barrier; both CTAs then arrive on the
@@ -1012,7 +1139,9 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
         const float lse_val = l > 0.f ? (m_ref + log2f(l)) * kLn2 : NEG_INF;
         inv_sm[tid] = l > 0.f ? 1.f / l : 0.f;
         if (leader && row < R) {
-          if (single)
+          if (single && SPARSE)  // query position (b / vq, b % vq), head row
+            p.lse[(static_cast<long long>(b / p.vq) * p.h_q + row) * p.vq + b % p.vq] = lse_val;
+          else if (single)
             p.lse[(static_cast<long long>(b) * p.h_q + row % p.h_q) * p.s_q + row / p.h_q] = lse_val;
           else
             p.lse_part[static_cast<long long>(split) * R + row] = lse_val;
@@ -1105,11 +1234,11 @@ __global__ void __launch_bounds__(PairCfg<FP8>::kThreads, 1)
 
 }  // namespace
 
-template <bool FP8>
+template <bool FP8, bool SPARSE = false>
 int launch_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_scale,
                 const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
-  using C = PairCfg<FP8>;
-  auto kern = mla_decode_pair_kernel<FP8>;
+  using C = PairCfg<FP8, SPARSE>;
+  auto kern = mla_decode_pair_kernel<FP8, SPARSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return static_cast<int>(e);
   cudaLaunchConfig_t cfg = {};
@@ -1136,6 +1265,10 @@ int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, c
 int launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
                            const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
   return launch_pair<true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
+}
+
+int launch_decode_pair_sparse_bf16(const CUtensorMap& tm_q, const DecodeParams& p, cudaStream_t stream) {
+  return launch_pair<false, true>(tm_q, tm_q, tm_q, tm_q, p, stream);
 }
 
 }  // namespace mla

@@ -83,6 +83,7 @@ int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, c
                             cudaStream_t stream);
 int launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
                            const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream);
+int launch_decode_pair_sparse_bf16(const CUtensorMap& tm_q, const DecodeParams& p, cudaStream_t stream);
 int launch_combine(const CombineParams& p, cudaStream_t stream);
 
 }  // namespace mla
