@@ -47,6 +47,8 @@
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
+#include <type_traits>
+
 #include "mla_internal.h"
 #include "mla_ptx.cuh"
 
@@ -82,6 +84,7 @@ constexpr int kOffQ = 0;
 constexpr int kOffP = kOffQ + kQBytes;
 constexpr int kOffSlots = kOffP + kPBytes;
 constexpr int kMiscBytes = 6144;
+constexpr int kRowSlots = 4;  // token-sparse: ring of row tables (one per pair step)
 constexpr int kTmemCols = 512;
 constexpr int kColO = 0;      // O^T dim block m at columns 128m
 constexpr int kColS = 256;    // S^T buffer sb at columns 256 + 128 sb
@@ -100,8 +103,8 @@ struct PairCfg {
   static constexpr int kOffRaw = kOffSlots + kNumSlots * kSlotBytes;
   static constexpr int kOffRope = kOffRaw + (FP8 ? kNumRaw * kRawBytes : 0);
   static constexpr int kOffMisc = kOffRope + kRopeBytes;
-  // token-sparse: + 1 KB for the row table of a step's 256 listed tokens
-  static constexpr int kMisc = kMiscBytes + (SPARSE ? 1024 : 0);
+  // token-sparse: + the ring of row tables, 1 KB per step (256 list slots)
+  static constexpr int kMisc = kMiscBytes + (SPARSE ? kRowSlots * 1024 : 0);
   static constexpr int kSmemBytes = kOffMisc + kMisc + 1024;  // + alignment slack
   static constexpr uint32_t kIdescQK = FP8 ? idesc_f16(256, kRows, false, false) : idesc_bf16(256, kRows, false, false);
   static constexpr uint32_t kIdescPV = FP8 ? idesc_f16(256, kRows, true, true) : idesc_bf16(256, kRows, true, true);
@@ -141,7 +144,9 @@ enum : int {
   // token-sparse, both: this CTA's gather warps' cp.async landed ([stages], then RoPE slot)
   kBarGather = kBarRopeReady + 1,
   kBarGatherRope = kBarGather + kMaxSlots,
-  kNumBars = kBarGatherRope + 1,
+  kBarRowFull = kBarGatherRope + 1,           // [row tables] token-sparse: the 32 lanes of the index warp
+  kBarRowEmpty = kBarRowFull + kRowSlots,     // [row tables] token-sparse: every gather lane
+  kNumBars = kBarRowEmpty + kRowSlots,
 };
 constexpr int kMiscHolder = 512;   // TMEM base address
 constexpr int kMiscAbort = 516;    // abort flag
@@ -154,8 +159,10 @@ constexpr int kMiscAlpha = 3584;   // float [128]
 constexpr int kMiscInv = 4096;     // float [128]
 constexpr int kMiscXMax = 4608;    // float [2][128]: the peer's block maxima
 constexpr int kMiscXL = 5632;      // float [128]: the peer's row sums
-constexpr int kMiscRowTab = 6144;  // token-sparse: int32 [256] cache rows of a step's listed tokens
-constexpr int kGatherThreads = 192;  // token-sparse: warps 10-15 copy the listed tokens' rows
+constexpr int kMiscRowTab = 6144;  // token-sparse: int32 [row tables][256] cache rows of a step's slots
+constexpr int kWarpIndex = 10;     // token-sparse: the warp that looks up the cache rows
+constexpr int kGatherWarps = 5;    // token-sparse: warps 11-15 copy the listed tokens' rows
+constexpr int kGatherThreads = 32 * kGatherWarps;
 static_assert(kNumBars * 8 <= kMiscHolder, "barrier area");
 static_assert(kMiscXL + 512 <= kMiscBytes, "misc area");
 
@@ -258,6 +265,12 @@ __device__ __forceinline__ bool warp_pwait(uint32_t bar, uint32_t parity, const 
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// every lane of the warp observes the phase itself (it then reads or overwrites what the phase
+// guards); false on every lane if any gave up
+__device__ __forceinline__ bool warp_all_wait(uint32_t bar, uint32_t parity, const PairCtl& c) {
+  return __all_sync(0xffffffffu, pwait(bar, parity, c) ? 1 : 0) != 0;
+}
+
 // Warp reduce-scatter (sum) of 64 column values over the 32 token lanes: afterwards lane l
 // holds the warp-wide sums of columns 2l and 2l + 1 in v[0], v[1].
 __device__ __forceinline__ void reduce_scatter64_sum(float* v, int lane) {
@@ -338,8 +351,9 @@ __device__ __forceinline__ void dequant_row(uint32_t src, uint32_t dst, uint32_t
 }
 
 // SPARSE (bf16 cache): token-sparse decode, every query position a request of topk listed
-// cache positions (see mla_decode.cu); warps 10-15 copy the listed tokens' rows into the stages
-// with 16-byte cp.async and the producer thread forwards each stage's completion to the leader.
+// cache positions (see mla_decode.cu): warp 10 looks up the cache rows of the listed positions
+// ahead of time, warps 11-15 copy those rows into the stages with 16-byte cp.async and the
+// producer thread forwards each stage's completion to the leader.
 template <bool FP8, bool SPARSE = false>
 __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
@@ -412,6 +426,10 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
     mbar_init(bar(kBarRopeReady), 2 * kDequantThreads / 32);
     for (int i = 0; i < kMaxSlots; ++i) mbar_init(bar(kBarGather + i), kGatherThreads);  // cp.async arrivals
     mbar_init(bar(kBarGatherRope), kGatherThreads);
+    for (int i = 0; i < kRowSlots; ++i) {
+      mbar_init(bar(kBarRowFull + i), 32);
+      mbar_init(bar(kBarRowEmpty + i), kGatherThreads);
+    }
     *abort_flag = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerFills) = 0;
     *reinterpret_cast<uint32_t*>(misc + kMiscPeerQ) = 0;
@@ -757,84 +775,117 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
       umma_commit_pair(bar(kBarDrain));
       drain_wait(bar(kBarDrain), 0);
     }
-  } else if (SPARSE && warp >= kWarpDequant) {
-    // ======================= gather warps (token-sparse, 10-15) ======================
-    // Per step group they look up the listed tokens' cache rows once (a shared table: K(t)
-    // this CTA's 128, V(t) the step's 256), then fill the RoPE slot and the stages in the fill
-    // order with 16-byte cp.async (two or four token rows per warp instruction, every sixth
-    // instruction per warp, zeros for empty slots).  Each lane's arrival on the CTA's gather
-    // barrier completes a stage once all its copies landed; the producer thread forwards that.
-    const int gt = threadIdx.x - kWarpDequant * 32;  // 0..191
-    const int gw = gt >> 5;
+  } else if (SPARSE && warp == kWarpIndex) {
+    // ======================= row lookups (token-sparse): one warp =======================
+    // For every pair step, ahead of the gather warps, the cache rows of the 256 list slots of its
+    // two blocks: lane l takes slots 4l .. 4l + 3 of each.  A slot names a key iff it is inside
+    // the list and holds a position in [0, L); its row is then page(position / 64) * 64 +
+    // position % 64 (or the position itself in a contiguous cache), else -1.
     int32_t* row_tab = reinterpret_cast<int32_t*>(misc + kMiscRowTab);
-    const char* kvb = static_cast<const char*>(p.kv);
-    uint32_t g = 0, rf = 0;
+    uint32_t st = 0;
     bool ok = true;
     ChunkWalk walk(p, part);
     int b, c0, c1, split;
-    bool aborted = false;
-    while (!aborted && walk.next(p, b, c0, c1, split)) {
+    while (ok && walk.next(p, b, c0, c1, split)) {
       const int breal = b / p.vq;
       const int L = p.cache_seqlens ? p.cache_seqlens[breal] : p.kv_len;
       const int32_t* bt = p.block_table ? p.block_table + static_cast<long long>(breal) * p.max_blocks : nullptr;
       const int32_t* ind = p.indices + static_cast<long long>(b) * p.topk;
       const int n = (c1 - c0 + 1) / 2;
-      // rows of nblk token blocks from kb0 (entry 128 q + r); false: some warp gave up (all see it)
-      auto table = [&](int kb0, int nblk) -> bool {
-        if (named_bar_any(3, kGatherThreads, !ok)) return false;  // also: the last group was issued
-        for (int e = gt; e < 128 * nblk; e += kGatherThreads) {
-          const int kb = kb0 + (e >> 7);
-          const int pos = kb * kBlockTokens + (e & 127);
-          const int idx = (kb < c1 && pos < p.topk) ? ind[pos] : -1;
-          row_tab[e] = (idx >= 0 && idx < L) ? (bt ? bt[idx >> 6] * kPage + (idx & (kPage - 1)) : idx) : -1;
+      for (int t = 0; t < n; ++t, ++st) {
+        if (!(ok = warp_all_wait(bar(kBarRowEmpty + st % kRowSlots), ((st / kRowSlots) & 1u) ^ 1u, wc))) break;
+        int r[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int kb = c0 + 2 * t + (q >> 2);
+          const int pos = kb * kBlockTokens + 4 * lane + (q & 3);
+          r[q] = (kb < c1 && pos < p.topk) ? ind[pos] : -1;
         }
-        named_bar_sync(3, kGatherThreads);
-        return true;
-      };
-      // the 128 rows of table entries tab0.. as natoms 64-dim columns from dims0: row i at
-      // dst + (i / 64) * pstride + (i % 64) * 128, column a at + a * hstride
-      auto copy = [&](uint32_t dst, int tab0, int dims0, int natoms, uint32_t pstride, uint32_t hstride) {
-        const int cpr = 8 * natoms, rpi = 32 / cpr;
-        const int sub = lane / cpr, c = lane % cpr;
-        const uint32_t a = static_cast<uint32_t>(c >> 3), cc = static_cast<uint32_t>(c & 7);
-        const char* src0 = kvb + (dims0 + 8 * c) * 2;
-        for (int it = gw; it < kBlockTokens / rpi; it += kGatherThreads / 32) {
-          const uint32_t i = static_cast<uint32_t>(it * rpi + sub);
-          const int row = row_tab[tab0 + static_cast<int>(i)];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int idx = r[q];
+          r[q] = (idx >= 0 && idx < L) ? (bt ? bt[idx >> 6] * kPage + (idx & (kPage - 1)) : idx) : -1;
+        }
+        int4* tab = reinterpret_cast<int4*>(row_tab + (st % kRowSlots) * 256 + 4 * lane);
+        tab[0] = make_int4(r[0], r[1], r[2], r[3]);
+        tab[32] = make_int4(r[4], r[5], r[6], r[7]);
+        mbar_arrive(bar(kBarRowFull + st % kRowSlots));
+      }
+    }
+  } else if (SPARSE && warp > kWarpIndex) {
+    // ======================= gather warps (token-sparse, 11-15) ======================
+    // They copy the stages in the fill order with 16-byte cp.async from the rows of the step's
+    // table (two or four token rows per warp instruction, every fifth instruction per warp, zeros
+    // for empty slots).  Each lane's arrival on the CTA's gather barrier completes a stage once
+    // all its copies landed; the producer thread forwards that to the leader.
+    const int gw = warp - kWarpIndex - 1;  // 0..4
+    const int32_t* row_tab = reinterpret_cast<const int32_t*>(misc + kMiscRowTab);
+    const char* kvb = static_cast<const char*>(p.kv);
+    uint32_t g = 0, rf = 0;
+    uint32_t steps = 0;  // row tables taken before this chunk
+    bool ok = true;
+    ChunkWalk walk(p, part);
+    int b, c0, c1, split;
+    // the 128 rows of table entries tab.. as natoms 64-dim columns from dims0: row i at
+    // dst + (i / 64) * pstride + (i % 64) * 128, column a at + a * hstride
+    // (all of this warp's table reads first, then its copies back to back)
+    auto copy = [&](uint32_t dst, const int32_t* tab, int dims0, auto natoms_c, uint32_t pstride, uint32_t hstride) {
+      constexpr int kCpr = 8 * decltype(natoms_c)::value, kRpi = 32 / kCpr, kInst = kBlockTokens / kRpi;
+      constexpr int kPerWarp = (kInst + kGatherWarps - 1) / kGatherWarps;
+      const int sub = lane / kCpr, c = lane % kCpr;
+      const uint32_t a = static_cast<uint32_t>(c >> 3), cc = static_cast<uint32_t>(c & 7);
+      const char* src0 = kvb + (dims0 + 8 * c) * 2;
+      int row[kPerWarp];
+#pragma unroll
+      for (int k = 0; k < kPerWarp; ++k) {
+        const int it = gw + k * kGatherWarps;
+        row[k] = it < kInst ? tab[it * kRpi + sub] : -1;
+      }
+#pragma unroll
+      for (int k = 0; k < kPerWarp; ++k) {
+        const int it = gw + k * kGatherWarps;
+        if (it < kInst) {
+          const uint32_t i = static_cast<uint32_t>(it * kRpi + sub);
           cp_async_16(dst + (i >> 6) * pstride + (i & 63u) * 128u + a * hstride + ((cc ^ (i & 7u)) << 4),
-                      src0 + (row >= 0 ? static_cast<long long>(row) * (kDqk * 2) : 0), row >= 0 ? 16u : 0u);
+                      src0 + (row[k] >= 0 ? static_cast<long long>(row[k]) * (kDqk * 2) : 0), row[k] >= 0 ? 16u : 0u);
         }
-      };
-      auto stage = [&](int tab0, int dims0, uint32_t pstride, uint32_t hstride) -> bool {
-        const uint32_t s = g % kNumSlots, use = g / kNumSlots;
-        if (!warp_pwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc, lane)) return false;
-        copy(sSlots + s * kSlotBytes, tab0, dims0, 2, pstride, hstride);
-        cp_async_arrive_noinc(bar(kBarGather + s));
-        ++g;
-        return true;
-      };
-      for (int e = 0; e < 2 * n; ++e) {
+      }
+    };
+    auto stage = [&](const int32_t* tab, int dims0, uint32_t pstride, uint32_t hstride) -> bool {
+      const uint32_t s = g % kNumSlots, use = g / kNumSlots;
+      if (!warp_all_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
+      copy(sSlots + s * kSlotBytes, tab, dims0, std::integral_constant<int, 2>{}, pstride, hstride);
+      cp_async_arrive_noinc(bar(kBarGather + s));
+      ++g;
+      return true;
+    };
+    while (ok && walk.next(p, b, c0, c1, split)) {
+      const int n = (c1 - c0 + 1) / 2;
+      for (int e = 0; ok && e < 2 * n; ++e) {
         bool is_v;
         int t;
         order_at(e, n, is_v, t);
+        const uint32_t st = steps + static_cast<uint32_t>(t);
+        const int32_t* tab = row_tab + (st % kRowSlots) * 256;  // [block a: 128][block b: 128]
         if (!is_v) {
-          if (!table(c0 + 2 * t + static_cast<int>(rank), 1)) { aborted = true; break; }
-          // RoPE dims of this CTA's block ([page][64 rows][64 dims]), then K stage j: dims
-          // 128j.. as [dim half][page][64 rows][64 dims]
-          if (ok) ok = warp_pwait(bar(kBarRopeEmpty), (rf & 1u) ^ 1u, wc, lane);
-          if (ok) {
-            copy(sRope, 0, kDv, 1, kBoxBytes, 0);
-            cp_async_arrive_noinc(bar(kBarGatherRope));
-            ++rf;
-          }
-          for (int j = 0; ok && j < kKFills; ++j) ok = stage(0, 128 * j, kBoxBytes, kHalfBytes);
+          // K(t): this CTA's block c0 + 2t + rank; the step's table is new here.  Its RoPE dims
+          // first ([page][64 rows][64 dims]), then K stage j: dims 128j.. as
+          // [dim half][page][64 rows][64 dims]
+          if (!(ok = warp_all_wait(bar(kBarRowFull + st % kRowSlots), (st / kRowSlots) & 1u, wc))) break;
+          const int32_t* kt = tab + 128 * static_cast<int>(rank);
+          if (!(ok = warp_all_wait(bar(kBarRopeEmpty), (rf & 1u) ^ 1u, wc))) break;
+          copy(sRope, kt, kDv, std::integral_constant<int, 1>{}, kBoxBytes, 0);
+          cp_async_arrive_noinc(bar(kBarGatherRope));
+          ++rf;
+          for (int j = 0; ok && j < kKFills; ++j) ok = stage(kt, 128 * j, kBoxBytes, kHalfBytes);
         } else {
-          if (!table(c0 + 2 * t, 2)) { aborted = true; break; }
           // V stage k = (m, blk): dims 256m + 128 rank.. of block blk as [page][dim half][64 rows]
           for (int k = 0; ok && k < kVFills; ++k)
-            ok = stage(128 * (k & 1), 256 * (k >> 1) + 128 * static_cast<int>(rank), kHalfBytes, kBoxBytes);
+            ok = stage(tab + 128 * (k & 1), 256 * (k >> 1) + 128 * static_cast<int>(rank), kHalfBytes, kBoxBytes);
+          if (ok) mbar_arrive(bar(kBarRowEmpty + st % kRowSlots));  // this lane has read the table
         }
       }
+      steps += static_cast<uint32_t>(n);
     }
     cp_async_wait_all();  // this lane's copies have landed before the CTA may exit
   } else if (FP8 && warp >= kWarpDequant) {
@@ -970,6 +1021,8 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
       for (int t = 0; t < n; ++t) {
         const int kb = c0 + 2 * t + static_cast<int>(rank);
         const int j = kb * kBlockTokens + tl;
+        // token-sparse: the position in list slot j, read before the wait for S hides its latency
+        const int sidx = (SPARSE && kb < c1 && j < p.topk) ? p.indices[static_cast<long long>(b) * p.topk + j] : -1;
         const int sb = static_cast<int>(u & 1u);
         bool ok = warp_pwait(bar(kBarSFull + sb), (u >> 1) & 1u, wc, lane);
         float x[64];
@@ -985,8 +1038,7 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
         int cmin = -(1 << 30);
         if constexpr (SPARSE) {
           // slot j of the list is a key iff it names a position in [0, L)
-          const int idx = (kb < c1 && j < p.topk) ? p.indices[static_cast<long long>(b) * p.topk + j] : -1;
-          if (idx < 0 || idx >= L) cmin = 1 << 30;
+          if (sidx < 0 || sidx >= L) cmin = 1 << 30;
         } else {
           if (p.causal) {
             const int i0 = j - L + p.s_q;
