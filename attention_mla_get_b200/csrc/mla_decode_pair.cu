@@ -1207,9 +1207,17 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
       tc_fence_after();
       {
         // O^T block h of this CTA: dim = lane's output dim, columns = query rows.  The tensor
-        // memory is released (OEmpty) as soon as the last load has landed, before its stores.
-        const int dim = 256 * h + 128 * static_cast<int>(rank) + tl;
-#pragma unroll
+        // memory is released (OEmpty) as soon as the last load has landed.  Each group of 32
+        // rows goes out through the P^T buffer (free once the chunk's last PV has completed):
+        // the softmax warps write it as [row][dim half][128 dims], then 64 of them copy one row
+        // half each to global memory with a bulk copy, which the TMA unit carries: plain
+        // stores from these warps took several times longer (they queue behind the traffic
+        // of the stage copies on the load/store path).
+        const uint32_t sStage = sP;
+        float* stage_f = reinterpret_cast<float*>(smem + kOffP);
+        __nv_bfloat16* stage_h = reinterpret_cast<__nv_bfloat16*>(smem + kOffP);
+        const bool issuer = tid < 64;  // row tid / 2 of the group, dim half tid % 2
+#pragma unroll 1
         for (int c = 0; c < kRows; c += 32) {
           float o[32];
           tmem_ld16(tmem + lane_base + kColO + 128u * h + c, o);
@@ -1220,18 +1228,38 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(lead(bar(kBarOEmpty)));
           }
+          if (c > 0) {
+            // the previous group's copies have read the buffer
+            if (issuer) bulk_wait_read_all();
+            named_bar_sync(1, kSoftmaxThreads);
+          }
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
+            const float val = o[e] * inv_sm[c + e];
+            const int k = e * 256 + h * 128 + tl;
+            if (single)
+              stage_h[k] = __float2bfloat16_rn(val);
+            else
+              stage_f[k] = val;
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, kSoftmaxThreads);
+          if (issuer) {
+            const int e = tid >> 1, hh = tid & 1;
             const int row = row0 + c + e;
             if (row < R) {
-              const float val = o[e] * inv_sm[c + e];
+              const int d0 = 256 * hh + 128 * static_cast<int>(rank);
+              const uint32_t k = static_cast<uint32_t>(e * 256 + hh * 128);
               if (single)
-                p.out[(static_cast<long long>(b) * R + row) * kDv + dim] = __float2bfloat16_rn(val);
+                bulk_store(p.out + (static_cast<long long>(b) * R + row) * kDv + d0, sStage + 2u * k, 256u);
               else
-                p.o_part[(static_cast<long long>(split) * R + row) * kDv + dim] = val;
+                bulk_store(p.o_part + (static_cast<long long>(split) * R + row) * kDv + d0, sStage + 4u * k, 512u);
             }
+            bulk_commit();
           }
         }
+        // the buffer is P^T again from the next step on (a softmax barrier comes first)
+        if (issuer) bulk_wait_read_all();
       }
       gchunk += static_cast<uint32_t>(kKFills + kVFills) * static_cast<uint32_t>(n);
       ++chunk;
