@@ -762,26 +762,59 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       const bool ok = warp_wait(bar(kBarOFull), chunk & 1, wc, lane);
       fail |= !ok;
       tc_fence_after();
+      {
+        // O^T block vs (dims 128 vs + tid), columns = query rows.  Groups of kGR rows go out
+        // through the P^T buffers (free once the chunk's last PV has completed): the softmax
+        // warps write them as [row][128 dims], then one thread per row copies the row to global
+        // memory with a bulk copy, which the TMA unit carries (plain stores from these warps
+        // were several times slower).
+        constexpr int kGR = (C::kNumP * C::kPBytes / 512) < RG ? (C::kNumP * C::kPBytes / 512) : RG;
+        float* stage_f = reinterpret_cast<float*>(smem + C::kOffP);
+        __nv_bfloat16* stage_h = reinterpret_cast<__nv_bfloat16*>(smem + C::kOffP);
+        bool first = true;
+#pragma unroll 1
+        for (int vs = 0; vs < 4; ++vs) {
+#pragma unroll 1
+          for (int g0 = 0; g0 < RG; g0 += kGR) {
+            if (!first) {
+              // the previous group's copies have read the buffers
+              if (tid < kGR) bulk_wait_read_all();
+              named_bar_sync(1, 128);
+            }
+            first = false;
 #pragma unroll
-      for (int vs = 0; vs < 4; ++vs) {
-        const int dim = vs * 128 + tid;
+            for (int c = 0; c < kGR; c += 16) {
+              float o[16];
+              tmem_ld16(tmem + lane_base + C::kColO + vs * RG + g0 + c, o);
+              tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < RG; c += 16) {
-          float o[16];
-          tmem_ld16(tmem + lane_base + C::kColO + vs * RG + c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int row = row0 + c + e;
-            if (row < R) {
-              const float val = o[e] * inv_sm[c + e];
-              if (single)
-                p.out[(static_cast<long long>(b) * R + row) * kDv + dim] = __float2bfloat16_rn(val);
-              else
-                p.o_part[(static_cast<long long>(split) * R + row) * kDv + dim] = val;
+              for (int e = 0; e < 16; ++e) {
+                const float val = o[e] * inv_sm[g0 + c + e];
+                if (single)
+                  stage_h[(c + e) * 128 + tid] = __float2bfloat16_rn(val);
+                else
+                  stage_f[(c + e) * 128 + tid] = val;
+              }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (tid < kGR) {
+              const int row = row0 + g0 + tid;
+              if (row < R) {
+                if (single)
+                  bulk_store(p.out + (static_cast<long long>(b) * R + row) * kDv + vs * 128,
+                             sP + static_cast<uint32_t>(tid) * 256u, 256u);
+                else
+                  bulk_store(p.o_part + (static_cast<long long>(split) * R + row) * kDv + vs * 128,
+                             sP + static_cast<uint32_t>(tid) * 512u, 512u);
+              }
+              bulk_commit();
             }
           }
         }
+        // the buffers hold P^T again from the next step on
+        if (tid < kGR) bulk_wait_read_all();
+        named_bar_sync(1, 128);
       }
       tc_fence_before();
       __syncwarp();
