@@ -39,6 +39,29 @@ struct WorkspaceLayout {
   size_t lse_off, o_off, total;
 };
 
+// The CTA-pair kernel's output maps (boxes of 128 dims x 32 rows, no swizzle): o_part fp32
+// {512, rows, batch + parts} in the workspace, out bf16 {512, rows, batch}.
+static bool encode_out_maps(EncodeTiledFn encode, mla::OutMaps* om, float* o_part, void* out, int rows, int batch,
+                            int parts) {
+  const cuuint32_t box[3] = {128, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDv), static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(batch) + static_cast<cuuint64_t>(parts)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDv) * 4, static_cast<cuuint64_t>(kDv) * 4 * rows};
+    if (encode(&om->o_part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, o_part, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDv), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(batch)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDv) * 2, static_cast<cuuint64_t>(kDv) * 2 * rows};
+  return encode(&om->out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 WorkspaceLayout workspace_layout(int batch, int parts, int rows) {
   const size_t splits = static_cast<size_t>(batch) + static_cast<size_t>(parts);
   WorkspaceLayout w;
@@ -193,10 +216,12 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   p.causal = causal ? 1 : 0;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
 
+  mla::OutMaps om;
+  if (pair && !encode_out_maps(encode, &om, p.o_part, out, rows, batch, num_sm_parts)) return MLA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = kv_dtype == MLA_KV_BF16 ? (pair ? mla::launch_decode_pair_bf16(tm_q, tm_kv, p, st)
+  int e = kv_dtype == MLA_KV_BF16 ? (pair ? mla::launch_decode_pair_bf16(tm_q, tm_kv, om, p, st)
                                           : mla::launch_decode_bf16(tm_q, tm_kv, p, rg, st))
-          : pair ? mla::launch_decode_pair_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, st)
+          : pair ? mla::launch_decode_pair_fp8(tm_q, tm_kv, tm_scale, tm_rope, om, p, st)
                  : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
 
@@ -291,8 +316,10 @@ int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_t num_bl
   p.indices = indices;
   p.topk = topk;
   p.vq = s_q;
+  mla::OutMaps om;
+  if (pair && !encode_out_maps(encode, &om, p.o_part, out, h_q, p.batch, num_sm_parts)) return MLA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, p, st) : mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
+  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, om, p, st) : mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
   mla::CombineParams cp{};
   cp.num_splits = num_splits;
@@ -363,8 +390,10 @@ int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const int32_t* i
   p.indices = indices;
   p.topk = topk;
   p.vq = s_q;
+  mla::OutMaps om;
+  if (pair && !encode_out_maps(encode, &om, p.o_part, out, h_q, p.batch, num_sm_parts)) return MLA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, p, st) : mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
+  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, om, p, st) : mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
   mla::CombineParams cp{};
   cp.num_splits = num_splits;

@@ -358,6 +358,7 @@ template <bool FP8, bool SPARSE = false>
 __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                            const __grid_constant__ CUtensorMap tm_scale, const __grid_constant__ CUtensorMap tm_rope,
+                           const __grid_constant__ CUtensorMap tm_opart, const __grid_constant__ CUtensorMap tm_out,
                            const DecodeParams p) {
   using C = PairCfg<FP8, SPARSE>;
   constexpr int kNumSlots = C::kNumSlots;
@@ -1209,14 +1210,13 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
         // O^T block h of this CTA: dim = lane's output dim, columns = query rows.  The tensor
         // memory is released (OEmpty) as soon as the last load has landed.  Each group of 32
         // rows goes out through the P^T buffer (free once the chunk's last PV has completed):
-        // the softmax warps write it as [row][dim half][128 dims], then 64 of them copy one row
-        // half each to global memory with a bulk copy, which the TMA unit carries: plain
-        // stores from these warps took several times longer (they queue behind the traffic
-        // of the stage copies on the load/store path).
+        // the softmax warps write it as [dim half][32 rows][128 dims], then one thread stores
+        // each half with a TMA tensor store (rows past the request's end fall outside the map).
+        // Plain stores from these warps took several times longer (they queue behind the
+        // traffic of the stage copies on the load/store path), and so did one bulk copy per row.
         const uint32_t sStage = sP;
         float* stage_f = reinterpret_cast<float*>(smem + kOffP);
         __nv_bfloat16* stage_h = reinterpret_cast<__nv_bfloat16*>(smem + kOffP);
-        const bool issuer = tid < 64;  // row tid / 2 of the group, dim half tid % 2
 #pragma unroll 1
         for (int c = 0; c < kRows; c += 32) {
           float o[32];
@@ -1229,14 +1229,14 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
             if (lane == 0) mbar_arrive_remote(lead(bar(kBarOEmpty)));
           }
           if (c > 0) {
-            // the previous group's copies have read the buffer
-            if (issuer) bulk_wait_read_all();
+            // the previous group's stores have read the buffer
+            if (tid == 0) bulk_wait_read_all();
             named_bar_sync(1, kSoftmaxThreads);
           }
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float val = o[e] * inv_sm[c + e];
-            const int k = e * 256 + h * 128 + tl;
+            const int k = h * 4096 + e * 128 + tl;
             if (single)
               stage_h[k] = __float2bfloat16_rn(val);
             else
@@ -1244,22 +1244,19 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
           }
           fence_proxy_async_smem();
           named_bar_sync(1, kSoftmaxThreads);
-          if (issuer) {
-            const int e = tid >> 1, hh = tid & 1;
-            const int row = row0 + c + e;
-            if (row < R) {
+          if (tid == 0) {
+            for (int hh = 0; hh < 2; ++hh) {
               const int d0 = 256 * hh + 128 * static_cast<int>(rank);
-              const uint32_t k = static_cast<uint32_t>(e * 256 + hh * 128);
               if (single)
-                bulk_store(p.out + (static_cast<long long>(b) * R + row) * kDv + d0, sStage + 2u * k, 256u);
+                tma_store_3d(&tm_out, sStage + hh * 8192u, d0, row0 + c, b);
               else
-                bulk_store(p.o_part + (static_cast<long long>(split) * R + row) * kDv + d0, sStage + 4u * k, 512u);
+                tma_store_3d(&tm_opart, sStage + hh * 16384u, d0, row0 + c, split);
             }
             bulk_commit();
           }
         }
         // the buffer is P^T again from the next step on (a softmax barrier comes first)
-        if (issuer) bulk_wait_read_all();
+        if (tid == 0) bulk_wait_read_all();
       }
       gchunk += static_cast<uint32_t>(kKFills + kVFills) * static_cast<uint32_t>(n);
       ++chunk;
@@ -1316,7 +1313,7 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
 
 template <bool FP8, bool SPARSE = false>
 int launch_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_scale,
-                const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
+                const CUtensorMap& tm_rope, const OutMaps& om, const DecodeParams& p, cudaStream_t stream) {
   using C = PairCfg<FP8, SPARSE>;
   auto kern = mla_decode_pair_kernel<FP8, SPARSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -1333,22 +1330,24 @@ int launch_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtenso
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_kv, tm_scale, tm_rope, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_kv, tm_scale, tm_rope, om.o_part, om.out, p);
   return static_cast<int>(e);
 }
 
-int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p,
-                            cudaStream_t stream) {
-  return launch_pair<false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const OutMaps& om,
+                            const DecodeParams& p, cudaStream_t stream) {
+  return launch_pair<false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
 }
 
 int launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
-                           const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
-  return launch_pair<true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
+                           const CUtensorMap& tm_rope, const OutMaps& om, const DecodeParams& p,
+                           cudaStream_t stream) {
+  return launch_pair<true>(tm_q, tm_codes, tm_scale, tm_rope, om, p, stream);
 }
 
-int launch_decode_pair_sparse_bf16(const CUtensorMap& tm_q, const DecodeParams& p, cudaStream_t stream) {
-  return launch_pair<false, true>(tm_q, tm_q, tm_q, tm_q, p, stream);
+int launch_decode_pair_sparse_bf16(const CUtensorMap& tm_q, const OutMaps& om, const DecodeParams& p,
+                                   cudaStream_t stream) {
+  return launch_pair<false, true>(tm_q, tm_q, tm_q, tm_q, om, p, stream);
 }
 
 }  // namespace mla
