@@ -39,11 +39,11 @@ struct WorkspaceLayout {
   size_t lse_off, o_off, total;
 };
 
-// The CTA-pair kernel's output maps (boxes of 128 dims x 32 rows, no swizzle): o_part fp32
+// The decode kernels' output maps (boxes of 128 dims x box_rows rows, no swizzle): o_part fp32
 // {512, rows, batch + parts} in the workspace, out bf16 {512, rows, batch}.
 static bool encode_out_maps(EncodeTiledFn encode, mla::OutMaps* om, float* o_part, void* out, int rows, int batch,
-                            int parts) {
-  const cuuint32_t box[3] = {128, 32, 1};
+                            int parts, int box_rows) {
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDv), static_cast<cuuint64_t>(rows),
@@ -217,12 +217,13 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
 
   mla::OutMaps om;
-  if (pair && !encode_out_maps(encode, &om, p.o_part, out, rows, batch, num_sm_parts)) return MLA_ERR_CUDA;
+  if (!encode_out_maps(encode, &om, p.o_part, out, rows, batch, num_sm_parts, rg == 16 ? 16 : 32))
+    return MLA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int e = kv_dtype == MLA_KV_BF16 ? (pair ? mla::launch_decode_pair_bf16(tm_q, tm_kv, om, p, st)
-                                          : mla::launch_decode_bf16(tm_q, tm_kv, p, rg, st))
+                                          : mla::launch_decode_bf16(tm_q, tm_kv, om, p, rg, st))
           : pair ? mla::launch_decode_pair_fp8(tm_q, tm_kv, tm_scale, tm_rope, om, p, st)
-                 : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, p, rg, st);
+                 : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, om, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
 
   mla::CombineParams cp{};
@@ -317,9 +318,11 @@ int mla_decode_kvcache_sparse(const void* q, const void* kvcache, int64_t num_bl
   p.topk = topk;
   p.vq = s_q;
   mla::OutMaps om;
-  if (pair && !encode_out_maps(encode, &om, p.o_part, out, h_q, p.batch, num_sm_parts)) return MLA_ERR_CUDA;
+  if (!encode_out_maps(encode, &om, p.o_part, out, h_q, p.batch, num_sm_parts, rg == 16 ? 16 : 32))
+    return MLA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, om, p, st) : mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
+  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, om, p, st)
+               : mla::launch_decode_sparse_bf16(tm_q, om, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
   mla::CombineParams cp{};
   cp.num_splits = num_splits;
@@ -391,9 +394,11 @@ int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const int32_t* i
   p.topk = topk;
   p.vq = s_q;
   mla::OutMaps om;
-  if (pair && !encode_out_maps(encode, &om, p.o_part, out, h_q, p.batch, num_sm_parts)) return MLA_ERR_CUDA;
+  if (!encode_out_maps(encode, &om, p.o_part, out, h_q, p.batch, num_sm_parts, rg == 16 ? 16 : 32))
+    return MLA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, om, p, st) : mla::launch_decode_sparse_bf16(tm_q, p, rg, st);
+  int e = pair ? mla::launch_decode_pair_sparse_bf16(tm_q, om, p, st)
+               : mla::launch_decode_sparse_bf16(tm_q, om, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;
   mla::CombineParams cp{};
   cp.num_splits = num_splits;

@@ -251,6 +251,7 @@ template <int RG, bool FP8, bool SPARSE = false>
 __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                       const __grid_constant__ CUtensorMap tm_scale, const __grid_constant__ CUtensorMap tm_rope,
+                      const __grid_constant__ CUtensorMap tm_opart, const __grid_constant__ CUtensorMap tm_out,
                       const DecodeParams p) {
   using C = Cfg<RG, FP8>;
   extern __shared__ uint8_t smem_raw[];
@@ -765,10 +766,11 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       {
         // O^T block vs (dims 128 vs + tid), columns = query rows.  Groups of kGR rows go out
         // through the P^T buffers (free once the chunk's last PV has completed): the softmax
-        // warps write them as [row][128 dims], then one thread per row copies the row to global
-        // memory with a bulk copy, which the TMA unit carries (plain stores from these warps
-        // were several times slower).
+        // warps write them as [row][128 dims], then one thread stores the group with a TMA
+        // tensor store (rows past the request's end fall outside the map).  Plain stores from
+        // these warps were slower.
         constexpr int kGR = (C::kNumP * C::kPBytes / 512) < RG ? (C::kNumP * C::kPBytes / 512) : RG;
+        static_assert(kGR == (RG == 16 ? 16 : 32), "output map box rows");
         float* stage_f = reinterpret_cast<float*>(smem + C::kOffP);
         __nv_bfloat16* stage_h = reinterpret_cast<__nv_bfloat16*>(smem + C::kOffP);
         bool first = true;
@@ -777,8 +779,8 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
 #pragma unroll 1
           for (int g0 = 0; g0 < RG; g0 += kGR) {
             if (!first) {
-              // the previous group's copies have read the buffers
-              if (tid < kGR) bulk_wait_read_all();
+              // the previous group's store has read the buffers
+              if (tid == 0) bulk_wait_read_all();
               named_bar_sync(1, 128);
             }
             first = false;
@@ -798,22 +800,17 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
             }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
-            if (tid < kGR) {
-              const int row = row0 + g0 + tid;
-              if (row < R) {
-                if (single)
-                  bulk_store(p.out + (static_cast<long long>(b) * R + row) * kDv + vs * 128,
-                             sP + static_cast<uint32_t>(tid) * 256u, 256u);
-                else
-                  bulk_store(p.o_part + (static_cast<long long>(split) * R + row) * kDv + vs * 128,
-                             sP + static_cast<uint32_t>(tid) * 512u, 512u);
-              }
+            if (tid == 0) {
+              if (single)
+                tma_store_3d(&tm_out, sP, vs * 128, row0 + g0, b);
+              else
+                tma_store_3d(&tm_opart, sP, vs * 128, row0 + g0, split);
               bulk_commit();
             }
           }
         }
         // the buffers hold P^T again from the next step on
-        if (tid < kGR) bulk_wait_read_all();
+        if (tid == 0) bulk_wait_read_all();
         named_bar_sync(1, 128);
       }
       tc_fence_before();
@@ -938,44 +935,46 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
 
 template <int RG, bool FP8, bool SPARSE = false>
 int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtensorMap& tm_scale,
-                const CUtensorMap& tm_rope, const DecodeParams& p, cudaStream_t stream) {
+                const CUtensorMap& tm_rope, const OutMaps& om, const DecodeParams& p, cudaStream_t stream) {
   using C = Cfg<RG, FP8>;
   auto kern = mla_decode_kernel<RG, FP8, SPARSE>;
   constexpr int kThreads = threads_of<RG, FP8, SPARSE>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid(p.num_sm_parts, p.row_groups, 1);
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, tm_scale, tm_rope, p);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, tm_scale, tm_rope, om.o_part, om.out, p);
   return static_cast<int>(cudaGetLastError());
 }
 
 }  // namespace
 
-int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, int rows_per_cta,
-                       cudaStream_t stream) {
+int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const OutMaps& om, const DecodeParams& p,
+                       int rows_per_cta, cudaStream_t stream) {
   switch (rows_per_cta) {
-    case 16: return launch_impl<16, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
-    case 32: return launch_impl<32, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
-    case 64: return launch_impl<64, false>(tm_q, tm_kv, tm_kv, tm_kv, p, stream);
+    case 16: return launch_impl<16, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
+    case 32: return launch_impl<32, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
+    case 64: return launch_impl<64, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }
 }
 
-int launch_decode_sparse_bf16(const CUtensorMap& tm_q, const DecodeParams& p, int rows_per_cta, cudaStream_t stream) {
+int launch_decode_sparse_bf16(const CUtensorMap& tm_q, const OutMaps& om, const DecodeParams& p, int rows_per_cta,
+                              cudaStream_t stream) {
   switch (rows_per_cta) {
-    case 16: return launch_impl<16, false, true>(tm_q, tm_q, tm_q, tm_q, p, stream);
-    case 32: return launch_impl<32, false, true>(tm_q, tm_q, tm_q, tm_q, p, stream);
-    case 64: return launch_impl<64, false, true>(tm_q, tm_q, tm_q, tm_q, p, stream);
+    case 16: return launch_impl<16, false, true>(tm_q, tm_q, tm_q, tm_q, om, p, stream);
+    case 32: return launch_impl<32, false, true>(tm_q, tm_q, tm_q, tm_q, om, p, stream);
+    case 64: return launch_impl<64, false, true>(tm_q, tm_q, tm_q, tm_q, om, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }
 }
 
 int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
-                      const CUtensorMap& tm_rope, const DecodeParams& p, int rows_per_cta, cudaStream_t stream) {
+                      const CUtensorMap& tm_rope, const OutMaps& om, const DecodeParams& p, int rows_per_cta,
+                      cudaStream_t stream) {
   switch (rows_per_cta) {
-    case 16: return launch_impl<16, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
-    case 32: return launch_impl<32, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
-    case 64: return launch_impl<64, true>(tm_q, tm_codes, tm_scale, tm_rope, p, stream);
+    case 16: return launch_impl<16, true>(tm_q, tm_codes, tm_scale, tm_rope, om, p, stream);
+    case 32: return launch_impl<32, true>(tm_q, tm_codes, tm_scale, tm_rope, om, p, stream);
+    case 64: return launch_impl<64, true>(tm_q, tm_codes, tm_scale, tm_rope, om, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }
 }

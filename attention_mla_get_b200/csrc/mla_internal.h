@@ -70,8 +70,8 @@ constexpr int kPairRows = 128;
 inline bool use_pair_kernel(int rows, bool /*fp8*/) { return rows > kRowsPerCta; }
 inline int sms_per_part(int rows) { return rows <= kRowsPerCta ? 1 : 2 * ((rows + kPairRows - 1) / kPairRows); }
 
-// Output tensor maps of the CTA-pair kernel's epilogue (TMA stores of 128 dims x 32 rows):
-// o_part fp32 {512, rows, splits}, out bf16 {512, rows, batch}
+// Output tensor maps of the decode kernels' epilogues (TMA stores of 128 dims x 32 rows, or 16
+// rows for the 16-row kernel): o_part fp32 {512, rows, splits}, out bf16 {512, rows, batch}
 struct OutMaps {
   CUtensorMap o_part;
   CUtensorMap out;
@@ -81,11 +81,13 @@ struct OutMaps {
 // cache_seqlens == nullptr: every one of the `batch` requests has uniform_len tokens
 int launch_scheduler(const int32_t* cache_seqlens, int batch, int num_sm_parts, int32_t* tile_md,
                      int32_t* num_splits, cudaStream_t stream, int uniform_len = 0);
-int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const DecodeParams& p, int rows_per_cta,
-                       cudaStream_t stream);
+int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const OutMaps& om, const DecodeParams& p,
+                       int rows_per_cta, cudaStream_t stream);
 int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
-                      const CUtensorMap& tm_rope, const DecodeParams& p, int rows_per_cta, cudaStream_t stream);
-int launch_decode_sparse_bf16(const CUtensorMap& tm_q, const DecodeParams& p, int rows_per_cta, cudaStream_t stream);
+                      const CUtensorMap& tm_rope, const OutMaps& om, const DecodeParams& p, int rows_per_cta,
+                      cudaStream_t stream);
+int launch_decode_sparse_bf16(const CUtensorMap& tm_q, const OutMaps& om, const DecodeParams& p, int rows_per_cta,
+                              cudaStream_t stream);
 int launch_decode_pair_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const OutMaps& om,
                             const DecodeParams& p, cudaStream_t stream);
 int launch_decode_pair_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
