@@ -12,8 +12,12 @@ value     KV bytes the step reads (exact token counts, 1152 B per bf16 token) pl
           and lse bytes, summed over all ranks, divided by the max-over-ranks device time
           (CUDA events on the launching stream).
 e2e       the same metric when every step also copies its inputs (q, block_table,
-          cache_seqlens) from pinned host memory and reads back out and lse; the KV cache
-          is resident device state, as in serving.
+          cache_seqlens, indices) from pinned host memory and reads back out and lse; the KV
+          cache is resident device state, as in serving.  The steps are pipelined as a
+          serving loop would run them: step k+1's inputs are copied in and step k-1's
+          results read back (two copy streams, double-buffered device inputs and outputs)
+          while step k computes; the timed region runs from before the first copy-in to
+          after the last read-back.
 roofline  the decode call (main kernel + combine), algorithmic bytes per launch divided by
           its mean CUDA-event duration, against the measured HBM copy bandwidth.
 cpu_baseline  the fp64 oracle timed on this host's cores on a bounded sample of requests.
@@ -297,16 +301,19 @@ def main():
                                                device=dev)
         return mla.mla_get_metadata(sl_, R, 1, num_sm_parts=parts)
 
-    def decode(q_, bt_, sl_, idx_, md, ns):
+    def decode_into(q_, bt_, sl_, idx_, md, ns, out_, lse_):
         if prefill:
-            mla.mla_sparse_prefill(q_, kv, idx_, case.softmax_scale, tile_md=md, num_splits=ns, out=out, lse=lse,
+            mla.mla_sparse_prefill(q_, kv, idx_, case.softmax_scale, tile_md=md, num_splits=ns, out=out_, lse=lse_,
                                    workspace=ws)
         elif sparse:
             mla.mla_decode_kvcache_sparse(q_, kv, bt_, sl_, idx_, 512, md, ns, softmax_scale=case.softmax_scale,
-                                          out=out, lse=lse, workspace=ws)
+                                          out=out_, lse=lse_, workspace=ws)
         else:
             mla.mla_decode_kvcache(q_, kv, bt_, sl_, 512, md, ns, softmax_scale=case.softmax_scale,
-                                   causal=case.causal, out=out, lse=lse, workspace=ws)
+                                   causal=case.causal, out=out_, lse=lse_, workspace=ws)
+
+    def decode(q_, bt_, sl_, idx_, md, ns):
+        decode_into(q_, bt_, sl_, idx_, md, ns, out, lse)
 
     def step():
         md, ns = metadata(sl)
@@ -348,32 +355,51 @@ def main():
     sl_h = sl.cpu().pin_memory()
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    q_d, bt_d, sl_d = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(sl)
     idx_h = idx.cpu().pin_memory() if sparse else None
-    idx_d = torch.empty_like(idx) if sparse else None
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4 + (idx_h.numel() * 4 if sparse else 0)
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    # double-buffered device inputs and outputs, two copy streams beside the compute stream
+    bufs = [dict(q=torch.empty_like(q), bt=torch.empty_like(bt), sl=torch.empty_like(sl),
+                 idx=torch.empty_like(idx) if sparse else None, out=torch.empty_like(out),
+                 lse=torch.empty_like(lse)) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        q_d.copy_(q_h, non_blocking=True)
-        bt_d.copy_(bt_h, non_blocking=True)
-        sl_d.copy_(sl_h, non_blocking=True)
-        if sparse:
-            idx_d.copy_(idx_h, non_blocking=True)
-        md, ns = metadata(sl_d)
-        decode(q_d, bt_d, sl_d, idx_d, md, ns)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+    def e2e_run(n):
+        computed = [torch.cuda.Event() for _ in range(n)]
+        out_read = [torch.cuda.Event() for _ in range(n)]
+        s_in.wait_stream(stream)  # nothing is copied in before the region starts
+        for k in range(n):
+            b = bufs[k % 2]
+            in_ready = torch.cuda.Event()
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(computed[k - 2])  # step k-2 has read these inputs
+                b["q"].copy_(q_h, non_blocking=True)
+                b["bt"].copy_(bt_h, non_blocking=True)
+                b["sl"].copy_(sl_h, non_blocking=True)
+                if sparse:
+                    b["idx"].copy_(idx_h, non_blocking=True)
+                in_ready.record(s_in)
+            stream.wait_event(in_ready)
+            if k >= 2:
+                stream.wait_event(out_read[k - 2])  # step k-2's results have been read back
+            md, ns = metadata(b["sl"])
+            decode_into(b["q"], b["bt"], b["sl"], b["idx"], md, ns, b["out"], b["lse"])
+            computed[k].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[k])
+                out_h.copy_(b["out"], non_blocking=True)
+                lse_h.copy_(b["lse"], non_blocking=True)
+                out_read[k].record(s_out)
+        stream.wait_event(out_read[n - 1])
 
     e2e_ms = None
     if not args.no_e2e:
-        for _ in range(args.warmup):
-            e2e_step()
+        e2e_run(args.warmup)
         barrier()
         s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s2.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        e2e_run(args.steps)
         t2.record(stream)
         barrier()
         e2e_ms = max_over_ranks(s2.elapsed_time(t2), world, dev)
