@@ -195,6 +195,7 @@ FP8_CASES = [
     ("fp8_r32", 2, 1, 32, [64, 777], False),
     ("fp8_r64", 2, 1, 64, [129, 1000], False),
     ("fp8_r128", 2, 1, 128, [130, 1000], False),
+    ("fp8_r96_pair_pad_rows", 2, 1, 96, [300, 64], False),
     ("fp8_r256_causal", 2, 2, 128, [3, 700], True),
 ]
 

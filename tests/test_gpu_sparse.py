@@ -29,6 +29,9 @@ CASES = [
     ("sp_r32_ragged_topk", 2, 1, 32, [129, 3000], 333, 0.0, 0.0),
     ("sp_r64", 2, 1, 64, [700, 1500], 300, 0.0, 0.05),
     ("sp_r128_two_groups", 2, 1, 128, [1000, 4000], 512, 0.05, 0.05),
+    # CTA pairs with a part-filled row group: rows past h_q are clipped by the output map
+    ("sp_r96_pair_pad_rows", 3, 1, 96, [700, 2000, 90], 384, 0.1, 0.0),
+    ("sp_r192_two_pairs", 2, 1, 192, [600, 1500], 300, 0.05, 0.05),
     ("sp_sq2_r48_pad_rows", 2, 2, 48, [400, 90], 160, 0.1, 0.0),
     ("sp_topk_over_L", 2, 1, 16, [40, 70], 256, 0.0, 0.0),
 ]
@@ -113,6 +116,7 @@ PREFILL_CASES = [
     ("pf_r16", 37, 16, 1000, 128, 0.1),
     ("pf_r64_ragged_kv", 64, 64, 777, 256, 0.0),
     ("pf_r128", 16, 128, 4096, 512, 0.05),
+    ("pf_r96_pair_pad_rows", 24, 96, 1500, 300, 0.1),
     ("pf_r32_many_tokens", 200, 32, 300, 64, 0.2),
 ]
 
