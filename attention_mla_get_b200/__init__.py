@@ -17,6 +17,10 @@ Calls (same names as the C-ABI):
     mla_decode_kvcache_sparse(q, kvcache, block_table, cache_seqlens, indices, d_v, tile_md,
                               num_splits, softmax_scale=None) -> (out bf16, lse fp32)
     mla_read_status(workspace, reset=False)
+    MLASession(batch, s_q, h_q, max_blocks, topk=0, kv_dtype=KV_BF16)     (mla_session_*)
+        .decode(q_host, kvcache, block_table_host, cache_seqlens_host, out_host, lse_host,
+                indices_host=None, softmax_scale=None, causal=False)    host buffers, pipelined
+        .join(), .status(reset=False), .close()
 
 The FlashMLA-style spellings of the usage examples on the pages are provided too:
 get_mla_metadata(cache_seqlens, s_q * h_q // h_kv, h_kv) and
@@ -79,6 +83,16 @@ def _load() -> ctypes.CDLL:
     lib.mla_sparse_prefill.restype = i32
     lib.mla_read_status.argtypes = [vp, i32, ctypes.POINTER(i32), vp]
     lib.mla_read_status.restype = i32
+    lib.mla_session_create.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]
+    lib.mla_session_create.restype = i32
+    lib.mla_session_decode.argtypes = [vp, vp, vp, i64, vp, vp, vp, ctypes.c_float, i32, vp, vp, vp]
+    lib.mla_session_decode.restype = i32
+    lib.mla_session_join.argtypes = [vp, vp]
+    lib.mla_session_join.restype = i32
+    lib.mla_session_status.argtypes = [vp, i32, ctypes.POINTER(i32)]
+    lib.mla_session_status.restype = i32
+    lib.mla_session_destroy.argtypes = [vp]
+    lib.mla_session_destroy.restype = i32
     lib.mla_strerror.argtypes = [i32]
     lib.mla_strerror.restype = ctypes.c_char_p
     lib.mla_version.argtypes = []
@@ -90,7 +104,8 @@ _lib = _load()
 
 EXPORTED = ("mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
             "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse", "mla_sparse_prefill",
-            "mla_read_status", "mla_strerror", "mla_version")
+            "mla_session_create", "mla_session_decode", "mla_session_join", "mla_session_status",
+            "mla_session_destroy", "mla_read_status", "mla_strerror", "mla_version")
 
 
 def mla_strerror(code: int) -> str:
@@ -315,3 +330,73 @@ __all__ = [
     "mla_strerror", "mla_version", "get_mla_metadata", "flash_mla_with_kvcache", "MLAError", "LIB_PATH",
     "KV_BF16", "KV_FP8",
 ]
+
+
+class MLASession:
+    """Decode steps with host (CPU, preferably pinned) inputs and outputs through the library's
+    serving session (mla_session_* in include/mla.h): the copies of step k + 1's inputs and of
+    step k - 1's outputs overlap step k on the GPU.  `decode` returns at once; call `join()`
+    and synchronise the stream before reading the host outputs."""
+
+    def __init__(self, batch: int, s_q: int, h_q: int, max_blocks: int, topk: int = 0, kv_dtype: int = KV_BF16,
+                 h_kv: int = 1, num_sm_parts: Optional[int] = None, device=None):
+        dev = torch.cuda.current_device() if device is None else torch.device(device).index
+        if num_sm_parts is None:
+            num_sm_parts = mla_num_sm_parts(h_q if topk > 0 else s_q * h_q, h_kv, dev)
+        handle = ctypes.c_void_p()
+        _check(_lib.mla_session_create(int(dev), int(batch), int(s_q), int(h_q), int(h_kv), int(max_blocks), int(topk),
+                                       int(kv_dtype), int(num_sm_parts), ctypes.byref(handle)), "mla_session_create")
+        self._h = handle
+        self.batch, self.s_q, self.h_q, self.max_blocks, self.topk = batch, s_q, h_q, max_blocks, topk
+        self.num_sm_parts = num_sm_parts
+
+    @staticmethod
+    def _host(t: torch.Tensor, dtype, numel: int, name: str) -> int:
+        if t.is_cuda or t.dtype != dtype or not t.is_contiguous() or t.numel() != numel:
+            raise ValueError(f"{name}: a contiguous host {dtype} tensor of {numel} elements is required")
+        return t.data_ptr()
+
+    def decode(self, q_host: torch.Tensor, kvcache: torch.Tensor, block_table_host: torch.Tensor,
+               cache_seqlens_host: torch.Tensor, out_host: torch.Tensor, lse_host: torch.Tensor,
+               indices_host: Optional[torch.Tensor] = None, softmax_scale: Optional[float] = None,
+               causal: bool = False, stream=None) -> None:
+        if self._h is None:
+            raise RuntimeError("session closed")
+        if not kvcache.is_cuda:
+            raise ValueError("kvcache must be a device tensor")
+        b, s_q, h_q = self.batch, self.s_q, self.h_q
+        positions = b * s_q
+        if softmax_scale is None:
+            softmax_scale = D_QK ** -0.5
+        num_blocks = kvcache.shape[0]
+        qp = self._host(q_host, torch.bfloat16, positions * h_q * D_QK, "q_host")
+        btp = self._host(block_table_host, torch.int32, b * self.max_blocks, "block_table_host")
+        slp = self._host(cache_seqlens_host, torch.int32, b, "cache_seqlens_host")
+        op = self._host(out_host, torch.bfloat16, positions * h_q * D_V, "out_host")
+        lp = self._host(lse_host, torch.float32, positions * h_q, "lse_host")
+        ip = None
+        if self.topk > 0:
+            if indices_host is None:
+                raise ValueError("indices_host is required in a token-sparse session")
+            ip = self._host(indices_host, torch.int32, positions * self.topk, "indices_host")
+        _check(_lib.mla_session_decode(self._h, qp, _ptr(kvcache), int(num_blocks), btp, slp, ip, float(softmax_scale),
+                                       1 if causal else 0, op, lp, _stream(stream)), "mla_session_decode")
+
+    def join(self, stream=None) -> None:
+        _check(_lib.mla_session_join(self._h, _stream(stream)), "mla_session_join")
+
+    def status(self, reset: bool = False) -> int:
+        v = ctypes.c_int(0)
+        _check(_lib.mla_session_status(self._h, 1 if reset else 0, ctypes.byref(v)), "mla_session_status")
+        return v.value
+
+    def close(self) -> None:
+        if self._h is not None:
+            h, self._h = self._h, None
+            _check(_lib.mla_session_destroy(h), "mla_session_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

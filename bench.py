@@ -13,11 +13,12 @@ value     KV bytes the step reads (exact token counts, 1152 B per bf16 token) pl
           (CUDA events on the launching stream).
 e2e       the same metric when every step also copies its inputs (q, block_table,
           cache_seqlens, indices) from pinned host memory and reads back out and lse; the KV
-          cache is resident device state, as in serving.  The steps are pipelined as a
-          serving loop would run them: step k+1's inputs are copied in and step k-1's
-          results read back (two copy streams, double-buffered device inputs and outputs)
-          while step k computes; the timed region runs from before the first copy-in to
-          after the last read-back.
+          cache is resident device state, as in serving.  Decode steps go through the
+          library's serving session (mla_session_decode with host buffers), which pipelines
+          them as a serving loop would: step k+1's inputs are copied in and step k-1's results
+          read back (two copy streams, double-buffered device staging) while step k computes;
+          sparse prefill, which has no session call, runs the same pipeline from Python.  The
+          timed region runs from before the first copy-in to after the last read-back.
 roofline  the decode call (main kernel + combine), algorithmic bytes per launch divided by
           its mean CUDA-event duration, against the measured HBM copy bandwidth.
 cpu_baseline  the fp64 oracle timed on this host's cores on a bounded sample of requests.
@@ -361,10 +362,23 @@ def main():
     # double-buffered device inputs and outputs, two copy streams beside the compute stream
     bufs = [dict(q=torch.empty_like(q), bt=torch.empty_like(bt), sl=torch.empty_like(sl),
                  idx=torch.empty_like(idx) if sparse else None, out=torch.empty_like(out),
-                 lse=torch.empty_like(lse)) for _ in range(2)]
+                 lse=torch.empty_like(lse)) for _ in range(2)] if prefill else None
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
+    session = None
+    if not prefill:
+        session = mla.MLASession(case.batch, case.s_q, case.h_q, case.block_table.shape[1],
+                                 topk=case.topk if sparse else 0,
+                                 kv_dtype=mla.KV_FP8 if case.kv_format == "fp8" else mla.KV_BF16,
+                                 num_sm_parts=parts)
+
     def e2e_run(n):
+        if session is not None:
+            for _ in range(n):
+                session.decode(q_h, kv, bt_h, sl_h, out_h, lse_h, indices_host=idx_h,
+                               softmax_scale=case.softmax_scale, causal=case.causal)
+            session.join()
+            return
         computed = [torch.cuda.Event() for _ in range(n)]
         out_read = [torch.cuda.Event() for _ in range(n)]
         s_in.wait_stream(stream)  # nothing is copied in before the region starts
@@ -403,6 +417,8 @@ def main():
         t2.record(stream)
         barrier()
         e2e_ms = max_over_ranks(s2.elapsed_time(t2), world, dev)
+    if session is not None:
+        session.close()
 
     if rank != 0:
         if world > 1:

@@ -23,8 +23,9 @@
  *
  * Conventions for every call
  *   - All pointers are DEVICE pointers unless stated otherwise; the caller owns every buffer.
- *   - The library allocates no device memory and never synchronises the stream; calls are
- *     enqueued on `stream` (a cudaStream_t, NULL = legacy default stream) and return at once.
+ *   - Outside the serving session (mla_session_*), the library allocates no device memory and
+ *     never synchronises the stream; calls are enqueued on `stream` (a cudaStream_t, NULL =
+ *     legacy default stream) and return at once.
  *   - Return value: MLA_OK (0) or a negative MLA_ERR_* code.  Argument errors are detected on
  *     the host before anything is enqueued.  A CUDA launch failure returns MLA_ERR_CUDA.
  *   - Values inside device arrays (seqlens, block_table) are trusted: out-of-range page ids are
@@ -193,6 +194,55 @@ MLA_API int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const in
                                int h_kv, int d_v, int topk, const int32_t* tile_md, int num_sm_parts,
                                const int32_t* num_splits, float softmax_scale, void* out, float* lse,
                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Serving session: decode steps whose inputs and outputs are HOST buffers (pinned memory lets
+ * the copies run asynchronously), pipelined two steps deep.  The one part of the library that
+ * allocates device memory and creates streams and events, all at mla_session_create: two sets
+ * of staging buffers (q, block_table, cache_seqlens, indices, out, lse), the tile metadata,
+ * the workspace, a copy-in and a copy-out stream.  The KV cache stays a device buffer of the
+ * caller.
+ *
+ * mla_session_create  device, batch, s_q, h_q, h_kv (= 1), max_blocks (block-table width),
+ *                     topk (0: dense decode; > 0: token-sparse decode, bf16 cache only, with
+ *                     indices [batch, s_q, topk] per step), kv_dtype, num_sm_parts (from
+ *                     mla_num_sm_parts(topk ? h_q : s_q * h_q, h_kv)).  *session receives the
+ *                     handle.  Argument errors as mla_decode_kvcache; MLA_ERR_CUDA if an
+ *                     allocation fails (nothing is left allocated).
+ * mla_session_decode  one step with host buffers: q [batch, s_q, h_q, 576] bf16,
+ *                     block_table [batch, max_blocks] and cache_seqlens [batch] int32, indices
+ *                     [batch, s_q, topk] int32 (token-sparse sessions; NULL otherwise),
+ *                     out [batch, s_q, h_q, 512] bf16 and lse [batch, h_q, s_q] fp32; kvcache
+ *                     as in mla_decode_kvcache.  Enqueues the copy of the inputs into staging set
+ *                     k % 2 (copy-in stream, after step k - 2 has read that set), the scheduler,
+ *                     decode and combine on `stream` (after that copy, and after step k - 2's
+ *                     results have been copied out), and the copy of out and lse into the host
+ *                     buffers (copy-out stream).  So step k + 1's copy-in and step k - 1's
+ *                     copy-out run while step k computes.  Returns at once; the host inputs
+ *                     must stay unchanged until the step's copy-in has run.
+ * mla_session_join    makes `stream` wait for the copy-out of every step enqueued so far (no
+ *                     host wait: synchronise `stream` to read the host outputs); the next step's
+ *                     copy-in is then ordered after the work enqueued on `stream` before it.
+ *                     The first step after mla_session_create is ordered the same way.
+ * mla_session_status  reads the session workspace's status word (MLA_STATUS_*) into *status
+ *                     after waiting for the session's work; reset != 0 clears it.
+ * mla_session_destroy waits for the session's work and frees everything it allocated.
+ */
+typedef struct mla_session mla_session;
+
+MLA_API int mla_session_create(int device, int batch, int s_q, int h_q, int h_kv, int max_blocks, int topk,
+                               int kv_dtype, int num_sm_parts, mla_session** session);
+
+MLA_API int mla_session_decode(mla_session* session, const void* q_host, const void* kvcache, int64_t num_blocks,
+                               const int32_t* block_table_host, const int32_t* cache_seqlens_host,
+                               const int32_t* indices_host, float softmax_scale, int causal, void* out_host,
+                               float* lse_host, void* stream);
+
+MLA_API int mla_session_join(mla_session* session, void* stream);
+
+MLA_API int mla_session_status(mla_session* session, int reset, int* status);
+
+MLA_API int mla_session_destroy(mla_session* session);
 
 /*
  * Reads the device status word of a workspace into *status (host pointer).  This call

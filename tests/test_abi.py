@@ -39,7 +39,8 @@ def test_every_declared_symbol_is_exported(lib):
     names = _declared()
     assert set(names) == {"mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
                           "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
-                          "mla_sparse_prefill",
+                          "mla_sparse_prefill", "mla_session_create", "mla_session_decode", "mla_session_join",
+                          "mla_session_status", "mla_session_destroy",
                           "mla_read_status", "mla_strerror", "mla_version"}
     so = os.path.join(ROOT, "attention_mla_get_b200", "libmla.so")
     nm = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True).stdout
@@ -144,3 +145,37 @@ def test_sparse_argument_errors_are_reported_before_any_launch(lib):
     assert g(2, 1, 0, 16, 1, fake, 4, fake, None) == -7
     assert g(2, 1, 64, 16, 2, fake, 4, fake, None) == -4
     assert g(2, 1, 64, 16, 1, fake, 0, fake, None) == -8
+
+
+def test_session_argument_errors(lib):
+    """mla_session_create checks its arguments before any CUDA call; without a usable device a
+    valid request fails with MLA_ERR_NO_DEVICE; the per-step calls reject a NULL session."""
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    lib.mla_session_create.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]
+    lib.mla_session_create.restype = i32
+    h = vp()
+    ref = ctypes.byref(h)
+    # device, batch, s_q, h_q, h_kv, max_blocks, topk, kv_dtype, num_sm_parts
+    assert lib.mla_session_create(0, 4, 1, 16, 1, 8, 0, 0, 74, None) == -1
+    assert lib.mla_session_create(0, 4, 1, 16, 2, 8, 0, 0, 74, ref) == -4      # h_kv != 1
+    assert lib.mla_session_create(0, 4, 1, 0, 1, 8, 0, 0, 74, ref) == -4       # h_q < 1
+    assert lib.mla_session_create(0, 4, 1, 16, 1, 8, 0, 7, 74, ref) == -5      # kv_dtype
+    assert lib.mla_session_create(0, 4, 1, 16, 1, 8, 64, 1, 74, ref) == -5     # sparse needs bf16
+    assert lib.mla_session_create(0, 0, 1, 16, 1, 8, 0, 0, 74, ref) == -7      # batch
+    assert lib.mla_session_create(0, 4, 1, 16, 1, 0, 0, 0, 74, ref) == -7      # max_blocks
+    assert lib.mla_session_create(0, 4, 1, 16, 1, 8, -1, 0, 74, ref) == -7     # topk < 0
+    assert lib.mla_session_create(0, 4, 64, 128, 1, 8, 0, 0, 74, ref) == -7    # 8192 rows
+    assert lib.mla_session_create(0, 4, 1, 16, 1, 8, 0, 0, 0, ref) == -8       # parts
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.mla_session_create(0, 4, 1, 16, 1, 8, 0, 0, 74, ref) == -9
+        assert not h.value
+    lib.mla_session_decode.argtypes = [vp] * 3 + [ctypes.c_int64] + [vp] * 3 + [ctypes.c_float, i32, vp, vp, vp]
+    lib.mla_session_decode.restype = i32
+    assert lib.mla_session_decode(None, 1, 1, 1, 1, 1, None, 1.0, 0, 1, 1, None) == -1
+    lib.mla_session_join.argtypes = [vp, vp]
+    assert lib.mla_session_join(None, None) == -1
+    lib.mla_session_status.argtypes = [vp, i32, ctypes.POINTER(i32)]
+    assert lib.mla_session_status(None, 0, ctypes.byref(i32())) == -1
+    lib.mla_session_destroy.argtypes = [vp]
+    assert lib.mla_session_destroy(None) == -1
