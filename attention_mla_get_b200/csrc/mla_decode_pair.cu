@@ -1233,14 +1233,19 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
             if (tid == 0) bulk_wait_read_all();
             named_bar_sync(1, kSoftmaxThreads);
           }
+          // the rows' 1 / l four at a time (one 16-byte load, the same for every lane)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float val = o[e] * inv_sm[c + e];
-            const int k = h * 4096 + e * 128 + tl;
-            if (single)
-              stage_h[k] = __float2bfloat16_rn(val);
-            else
-              stage_f[k] = val;
+          for (int e = 0; e < 32; e += 4) {
+            const float4 iv = *reinterpret_cast<const float4*>(inv_sm + c + e);
+            const float v[4] = {o[e] * iv.x, o[e + 1] * iv.y, o[e + 2] * iv.z, o[e + 3] * iv.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int k = h * 4096 + (e + j) * 128 + tl;
+              if (single)
+                stage_h[k] = __float2bfloat16_rn(v[j]);
+              else
+                stage_f[k] = v[j];
+            }
           }
           fence_proxy_async_smem();
           named_bar_sync(1, kSoftmaxThreads);
