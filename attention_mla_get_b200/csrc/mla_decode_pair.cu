@@ -1210,12 +1210,15 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
         // O^T block h of this CTA: dim = lane's output dim, columns = query rows.  The tensor
         // memory is released (OEmpty) as soon as the last load has landed.  Each group of 32
         // rows goes out through the P^T buffer (free once the chunk's last PV has completed):
-        // the softmax warps write it as [dim half][32 rows][128 dims], then one thread stores
-        // each half with a TMA tensor store (rows past the request's end fall outside the map).
+        // the softmax warps write it as [dim half][32 rows][128 dims], then a TMA tensor store
+        // per half writes it out (rows past the request's end fall outside the map).
         // Plain stores from these warps took several times longer (they queue behind the
         // traffic of the stage copies on the load/store path), and so did one bulk copy per row.
         const uint32_t sStage = sP;
         float* stage_f = reinterpret_cast<float*>(smem + kOffP);
+        // thread 0 stores dim half 0, thread 32 (another warp) dim half 1; FP8: thread 0 both
+        // (the second issuer's registers cost the FP8 kernel more than it gains)
+        const int issuer = tid == 0 ? 0 : (!FP8 && tid == 32 ? 1 : -1);
         __nv_bfloat16* stage_h = reinterpret_cast<__nv_bfloat16*>(smem + kOffP);
 #pragma unroll 1
         for (int c = 0; c < kRows; c += 32) {
@@ -1230,7 +1233,7 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
           }
           if (c > 0) {
             // the previous group's stores have read the buffer
-            if (tid == 0) bulk_wait_read_all();
+            if (issuer >= 0) bulk_wait_read_all();
             named_bar_sync(1, kSoftmaxThreads);
           }
           // the rows' 1 / l four at a time (one 16-byte load, the same for every lane)
@@ -1249,8 +1252,8 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
           }
           fence_proxy_async_smem();
           named_bar_sync(1, kSoftmaxThreads);
-          if (tid == 0) {
-            for (int hh = 0; hh < 2; ++hh) {
+          if (issuer >= 0) {
+            for (int hh = issuer; hh < 2; hh += FP8 ? 1 : 2) {
               const int d0 = 256 * hh + 128 * static_cast<int>(rank);
               if (single)
                 tma_store_3d(&tm_out, sStage + hh * 8192u, d0, row0 + c, b);
@@ -1261,7 +1264,7 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
           }
         }
         // the buffer is P^T again from the next step on (a softmax barrier comes first)
-        if (tid == 0) bulk_wait_read_all();
+        if (issuer >= 0) bulk_wait_read_all();
       }
       gchunk += static_cast<uint32_t>(kKFills + kVFills) * static_cast<uint32_t>(n);
       ++chunk;
