@@ -327,6 +327,9 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
   const uint32_t tmem = *tmem_holder;
 
   pdl_launch_dependents();
+  // launched as a programmatic dependent of the tile scheduler: the set-up above overlapped
+  // it; its metadata is complete and visible from here on
+  pdl_wait_primary();
 
   if (SPARSE && (warp == 4 || warp >= 6)) {
     // ======================= gather producers (token-sparse) =======================
@@ -941,9 +944,18 @@ int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtenso
   constexpr int kThreads = threads_of<RG, FP8, SPARSE>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return static_cast<int>(e);
-  dim3 grid(p.num_sm_parts, p.row_groups, 1);
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, tm_scale, tm_rope, om.o_part, om.out, p);
-  return static_cast<int>(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.num_sm_parts, p.row_groups, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlaps the scheduler's tail
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_kv, tm_scale, tm_rope, om.o_part, om.out, p);
+  return static_cast<int>(e);
 }
 
 }  // namespace

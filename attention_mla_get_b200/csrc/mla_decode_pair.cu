@@ -456,6 +456,9 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   pdl_launch_dependents();
+  // launched as a programmatic dependent of the tile scheduler: the set-up above overlapped
+  // it; its metadata is complete and visible from here on
+  pdl_wait_primary();
 
   // state the exit sequence needs
   uint32_t fills = 0;  // producer: stage fills issued
@@ -1331,13 +1334,15 @@ int launch_pair(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtenso
   cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlaps the scheduler's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_kv, tm_scale, tm_rope, om.o_part, om.out, p);
   return static_cast<int>(e);
 }

@@ -16,6 +16,7 @@
 // metadata in a few microseconds: a scan of costs, a binary search per part, a scan of
 // chunk counts.
 #include "mla_internal.h"
+#include "mla_ptx.cuh"
 
 namespace mla {
 
@@ -63,6 +64,7 @@ __global__ void __launch_bounds__(kSchedThreads)
   const long long F = kFixedSplitCost;
   const int tid = threadIdx.x;
   const bool on_chip = batch <= kSmemBatch;
+  pdl_launch_dependents();  // the decode kernel's set-up may start now; it waits for this grid
 
   // pass 1: ns[b + 1] = C_{b+1} (inclusive prefix of costs), T
   long long carry = 0;
