@@ -173,7 +173,7 @@ def oracle_baseline(case, budget_s: float = 15.0):
 # DRAM bytes (read + write) per launch of the main kernel from an ncu capture of the current
 # kernel, scaled to the full workload by the KV bytes it processes (see profiles/); None when
 # the kernel has changed since the counters were taken.
-TRAFFIC = {"mem_b128_h16_L8192": 1255.4e6}
+TRAFFIC = {"mem_b128_h16_L8192": 1253.8e6}
 
 
 def rank_case(workload: str, rank: int, batch=None):
