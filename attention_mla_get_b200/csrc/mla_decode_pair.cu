@@ -1,5 +1,5 @@
-// Split-KV MLA decode on CTA pairs (cta_group::2) for requests with more than 64 query rows,
-// bf16 paged KV cache.
+// Split-KV MLA decode on CTA pairs (cta_group::2) for requests with more than 64 query rows:
+// bf16 or FP8 paged KV cache, and token-sparse decode / sparse prefill (bf16).
 //
 // The problem is the one of mla_decode.cu (FlashMLA pages: mha_fwd_kvcache_mla on a paged
 // latent cache of 576-dim tokens, V = the first 512 dims, 64-token pages addressed by
@@ -37,12 +37,19 @@
 //
 // FP8 cache (656-byte tokens: 512 e4m3 codes, 4 fp32 scales per 128 dims, 64 bf16 RoPE dims;
 // the wmrh.cn page, "FP8 KV缓存内存效率" table): the producer TMA-loads raw code columns (128
-// dims x 2 pages) with their scales into a raw ring of this CTA; two dequant warps write each
+// dims x 2 pages) with their scales into a raw ring of this CTA; four dequant warps write each
 // stage of the same order as f16 (code * scale) into the 32 KB stages, with zeros for tokens
 // outside the request, and convert the Q tile and each RoPE slot from bf16 to f16 in place.
 // The MMAs then run on f16 operands: e4m3 codes are exact in f16, which also keeps 11
 // mantissa bits of q, P and code * scale where bf16 keeps 8 (f16's range, |x| < 65504, holds
 // for the scaled cache and the queries).
+//
+// Token-sparse (SPARSE): the steps run over 128-slot blocks of each query position's index
+// list; a row-lookup warp and five gather warps copy the listed rows with 16-byte cp.async.
+//
+// Epilogue: each 32-row group of O^T goes from tensor memory through the P^T buffer to global
+// memory with TMA tensor stores.  The kernel is launched as a programmatic dependent of the
+// tile scheduler: its set-up overlaps the scheduler, and it waits for the metadata after it.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math_constants.h>
