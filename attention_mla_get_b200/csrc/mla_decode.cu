@@ -38,6 +38,11 @@
 // bf16 into the same swizzled slot ring the MMA reads (same order as above), and TMA-loads the
 // RoPE dims straight into their slot with the 128-byte swizzle.  Tokens past the end of the
 // request are written as zeros, so no tail fix-up is needed.
+//
+// Token-sparse decode (SPARSE, bf16): seven gather warps copy the listed tokens' rows into the
+// slots with 16-byte cp.async (see the kernel's gather branch).  The epilogue writes each group
+// of rows of O^T through the P^T buffers with a TMA tensor store, and the kernel is launched as
+// a programmatic dependent of the tile scheduler (set-up first, then it waits for the metadata).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math_constants.h>
