@@ -27,7 +27,8 @@ constexpr int kSmemBatch = 8192;  // batches up to this size keep the prefix arr
 
 __device__ __forceinline__ long long blocks_of(int L) { return L > 0 ? (L + kBlockTokens - 1) / kBlockTokens : 0; }
 
-// Inclusive scan of v over the CTA; returns the thread's inclusive prefix, *total gets the sum.
+// Inclusive scan of v over the CTA (any multiple of 32 threads up to 1024); returns the
+// thread's inclusive prefix, *total gets the sum.
 __device__ long long block_scan(long long v, long long* warp_tot, long long* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -38,7 +39,7 @@ __device__ long long block_scan(long long v, long long* warp_tot, long long* tot
   if (lane == 31) warp_tot[warp] = v;
   __syncthreads();
   if (warp == 0) {
-    long long w = warp_tot[lane];
+    long long w = lane < static_cast<int>(blockDim.x >> 5) ? warp_tot[lane] : 0;  // absent warps: 0
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const long long u = __shfl_up_sync(0xffffffffu, w, o);
@@ -66,11 +67,14 @@ __global__ void __launch_bounds__(kSchedThreads)
   const bool on_chip = batch <= kSmemBatch;
   pdl_launch_dependents();  // the decode kernel's set-up may start now; it waits for this grid
 
+  const int nthreads = static_cast<int>(blockDim.x);
   // pass 1: ns[b + 1] = C_{b+1} (inclusive prefix of costs), T
   long long carry = 0;
-  for (int base = 0; base < batch; base += kSchedThreads) {
+  long long n_first = 0;  // this thread's cost in the first tile (reused by pass 3 when it is the only one)
+  for (int base = 0; base < batch; base += nthreads) {
     const int b = base + tid;
     const long long n = b < batch ? blocks_of(seqlens ? seqlens[b] : uniform_len) : 0;
+    if (base == 0) n_first = n;
     long long tile_total;
     const long long incl = block_scan(n > 0 ? n + F : 0, warp_tot, &tile_total) + carry;
     if (b < batch) {
@@ -105,7 +109,7 @@ __global__ void __launch_bounds__(kSchedThreads)
     const long long j = x - (cb + F);
     fj = j > 0 ? static_cast<int>(j) : 0;
   };
-  for (int p = tid; p < parts; p += kSchedThreads) {
+  for (int p = tid; p < parts; p += nthreads) {
     int bb, bj, eb, ej;
     find(static_cast<long long>(p) * q, bb, bj);
     find(static_cast<long long>(p + 1) * q, eb, ej);
@@ -128,9 +132,9 @@ __global__ void __launch_bounds__(kSchedThreads)
   // because ns is overwritten here)
   carry = 0;
   long long chunk_carry = 0;
-  for (int base = 0; base < batch; base += kSchedThreads) {
+  for (int base = 0; base < batch; base += nthreads) {
     const int b = base + tid;
-    const long long n = b < batch ? blocks_of(seqlens ? seqlens[b] : uniform_len) : 0;
+    const long long n = batch <= nthreads ? n_first : (b < batch ? blocks_of(seqlens ? seqlens[b] : uniform_len) : 0);
     long long tile_total;
     const long long incl = block_scan(n > 0 ? n + F : 0, warp_tot, &tile_total) + carry;
     const long long cb = incl - (n > 0 ? n + F : 0);
@@ -144,7 +148,7 @@ __global__ void __launch_bounds__(kSchedThreads)
   __syncthreads();
 
   // pass 4: absolute split index of each part's first chunk
-  for (int p = tid; p < parts; p += kSchedThreads) {
+  for (int p = tid; p < parts; p += nthreads) {
     int32_t* row = md + static_cast<long long>(p) * kMdInts;
     row[4] += ns[row[0]];
   }
@@ -154,8 +158,12 @@ __global__ void __launch_bounds__(kSchedThreads)
 
 int launch_scheduler(const int32_t* cache_seqlens, int batch, int num_sm_parts, int32_t* tile_md,
                      int32_t* num_splits, cudaStream_t stream, int uniform_len) {
-  mla_tile_scheduler_kernel<<<1, kSchedThreads, 0, stream>>>(cache_seqlens, uniform_len, batch, num_sm_parts,
-                                                             tile_md, num_splits);
+  // one thread per request (and per part), in whole warps, at most kSchedThreads: small batches
+  // take fewer, cheaper barriers
+  const int want = batch > num_sm_parts ? batch : num_sm_parts;
+  const int threads = want >= kSchedThreads ? kSchedThreads : (want < 32 ? 32 : (want + 31) / 32 * 32);
+  mla_tile_scheduler_kernel<<<1, threads, 0, stream>>>(cache_seqlens, uniform_len, batch, num_sm_parts, tile_md,
+                                                       num_splits);
   return static_cast<int>(cudaGetLastError());
 }
 
