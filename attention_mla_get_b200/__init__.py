@@ -81,6 +81,8 @@ def _load() -> ctypes.CDLL:
     lib.mla_sparse_prefill.argtypes = [vp, vp, i32, vp, i32, i32, i32, i32, i32, vp, i32, vp, ctypes.c_float, vp, vp,
                                        vp, sz, vp]
     lib.mla_sparse_prefill.restype = i32
+    lib.mla_fault_injection_arm.argtypes = [ctypes.c_longlong, i32]
+    lib.mla_fault_injection_arm.restype = i32
     lib.mla_read_status.argtypes = [vp, i32, ctypes.POINTER(i32), vp]
     lib.mla_read_status.restype = i32
     lib.mla_session_create.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]
@@ -103,9 +105,9 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 
 EXPORTED = ("mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-            "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse", "mla_sparse_prefill",
+            "mla_decode_kvcache_noalloc", "mla_noalloc_read_status", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse", "mla_sparse_prefill",
             "mla_session_create", "mla_session_decode", "mla_session_join", "mla_session_status",
-            "mla_session_destroy", "mla_read_status", "mla_strerror", "mla_version")
+            "mla_session_destroy", "mla_read_status", "mla_fault_injection_arm", "mla_strerror", "mla_version")
 
 
 def mla_strerror(code: int) -> str:
@@ -131,6 +133,33 @@ def _stream(stream) -> int:
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
+
+
+def _require(t, name: str, dtype, ndim: Optional[int] = None, shape=None) -> None:
+    """dtype / rank / shape check of one tensor argument (before any device check, so that a
+    wrong dtype is reported as such whatever the device)."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _on_device(device, **tensors) -> None:
+    """Every tensor argument is CUDA-resident on `device` and contiguous (the library reads
+    raw row-major device memory)."""
+    if device.type != "cuda":
+        raise ValueError(f"{next(iter(tensors))} must be a CUDA tensor, got {device}")
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda or t.device != device:
+            raise ValueError(f"{name} must be a CUDA tensor on {device}, got {t.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
 
 
 def mla_num_sm_parts(rows_per_kv_head: int, h_kv: int = 1, device=None) -> int:
@@ -168,26 +197,41 @@ def mla_decode_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torc
                        lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                        stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """MLA decode: returns (out bf16 [b, s_q, h_q, 512], lse fp32 [b, h_q, s_q])."""
-    if q.dtype != torch.bfloat16 or q.dim() != 4 or q.shape[-1] != D_QK:
+    _require(q, "q", torch.bfloat16, 4)
+    if q.shape[-1] != D_QK:
         raise ValueError("q must be bf16 [batch, s_q, h_q, 576]")
-    if not q.is_contiguous():
-        q = q.contiguous()
     b, s_q, h_q, _ = q.shape
     if kv_dtype is None:
         kv_dtype = KV_FP8 if kvcache.dtype == torch.uint8 else KV_BF16
     if kv_dtype == KV_BF16:
-        if kvcache.dtype != torch.bfloat16 or kvcache.shape[1] != PAGE or kvcache.shape[-1] != D_QK:
+        if kvcache.dtype != torch.bfloat16 or kvcache.dim() not in (3, 4) or kvcache.shape[1] != PAGE or \
+                kvcache.shape[-1] != D_QK:
             raise ValueError("bf16 kvcache must be [num_blocks, 64, (1,) 576]")
-        h_kv = kvcache.shape[2] if kvcache.dim() == 4 else 1
-    else:
-        if kvcache.dtype != torch.uint8 or kvcache.shape[1] != PAGE or kvcache.shape[-1] != FP8_TOKEN_BYTES:
+    elif kv_dtype == KV_FP8:
+        if kvcache.dtype != torch.uint8 or kvcache.dim() not in (3, 4) or kvcache.shape[1] != PAGE or \
+                kvcache.shape[-1] != FP8_TOKEN_BYTES:
             raise ValueError("fp8 kvcache must be uint8 [num_blocks, 64, (1,) 656]")
-        h_kv = kvcache.shape[2] if kvcache.dim() == 4 else 1
-    if not kvcache.is_contiguous():
-        raise ValueError("kvcache must be contiguous")
-    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != b:
+    else:
+        raise ValueError("kv_dtype must be KV_BF16 or KV_FP8")
+    h_kv = kvcache.shape[2] if kvcache.dim() == 4 else 1
+    _require(block_table, "block_table", torch.int32, 2)
+    if block_table.shape[0] != b:
         raise ValueError("block_table must be int32 [batch, max_blocks]")
-    block_table = block_table.contiguous()
+    _require(cache_seqlens, "cache_seqlens", torch.int32, shape=(b,))
+    _require(tile_md, "tile_md", torch.int32, 2)
+    if tile_md.shape[1] != 8 or tile_md.shape[0] < 1:
+        raise ValueError("tile_md must be int32 [num_sm_parts, 8] from mla_get_metadata")
+    _require(num_splits, "num_splits", torch.int32, shape=(b + 1,))
+    if out is not None:
+        _require(out, "out", torch.bfloat16, shape=(b, s_q, h_q, D_V))
+    if lse is not None:
+        _require(lse, "lse", torch.float32, shape=(b, h_q, s_q))
+    if workspace is not None:
+        _require(workspace, "workspace", torch.uint8)
+    q = q.contiguous() if q.is_cuda else q
+    block_table = block_table.contiguous() if block_table.is_cuda else block_table
+    _on_device(q.device, q=q, kvcache=kvcache, block_table=block_table, cache_seqlens=cache_seqlens,
+               tile_md=tile_md, num_splits=num_splits, out=out, lse=lse, workspace=workspace)
     if softmax_scale is None:
         softmax_scale = D_QK ** -0.5
     rows = s_q * h_q // max(1, h_kv)
@@ -231,21 +275,35 @@ def mla_decode_kvcache_sparse(q: torch.Tensor, kvcache: torch.Tensor, block_tabl
                               stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Token-sparse MLA decode over indices int32 [b, s_q, topk] (bf16 cache):
     returns (out bf16 [b, s_q, h_q, 512], lse fp32 [b, h_q, s_q])."""
-    if q.dtype != torch.bfloat16 or q.dim() != 4 or q.shape[-1] != D_QK:
+    _require(q, "q", torch.bfloat16, 4)
+    if q.shape[-1] != D_QK:
         raise ValueError("q must be bf16 [batch, s_q, h_q, 576]")
-    q = q.contiguous()
     b, s_q, h_q, _ = q.shape
-    if kvcache.dtype != torch.bfloat16 or kvcache.shape[1] != PAGE or kvcache.shape[-1] != D_QK:
+    if kvcache.dtype != torch.bfloat16 or kvcache.dim() not in (3, 4) or kvcache.shape[1] != PAGE or \
+            kvcache.shape[-1] != D_QK:
         raise ValueError("kvcache must be bf16 [num_blocks, 64, (1,) 576] (token-sparse decode reads bf16 caches)")
-    if not kvcache.is_contiguous():
-        raise ValueError("kvcache must be contiguous")
     h_kv = kvcache.shape[2] if kvcache.dim() == 4 else 1
-    if indices.dtype != torch.int32 or indices.dim() != 3 or tuple(indices.shape[:2]) != (b, s_q):
+    _require(indices, "indices", torch.int32, 3)
+    if tuple(indices.shape[:2]) != (b, s_q):
         raise ValueError("indices must be int32 [batch, s_q, topk]")
-    indices = indices.contiguous()
-    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != b:
+    _require(block_table, "block_table", torch.int32, 2)
+    if block_table.shape[0] != b:
         raise ValueError("block_table must be int32 [batch, max_blocks]")
-    block_table = block_table.contiguous()
+    _require(cache_seqlens, "cache_seqlens", torch.int32, shape=(b,))
+    _require(tile_md, "tile_md", torch.int32, 2)
+    if tile_md.shape[1] != 8 or tile_md.shape[0] < 1:
+        raise ValueError("tile_md must be int32 [num_sm_parts, 8] from mla_get_metadata_sparse")
+    _require(num_splits, "num_splits", torch.int32, shape=(b * s_q + 1,))
+    if out is not None:
+        _require(out, "out", torch.bfloat16, shape=(b, s_q, h_q, D_V))
+    if lse is not None:
+        _require(lse, "lse", torch.float32, shape=(b, h_q, s_q))
+    if workspace is not None:
+        _require(workspace, "workspace", torch.uint8)
+    if q.is_cuda:
+        q, indices, block_table = q.contiguous(), indices.contiguous(), block_table.contiguous()
+    _on_device(q.device, q=q, kvcache=kvcache, block_table=block_table, cache_seqlens=cache_seqlens,
+               indices=indices, tile_md=tile_md, num_splits=num_splits, out=out, lse=lse, workspace=workspace)
     topk = indices.shape[2]
     if softmax_scale is None:
         softmax_scale = D_QK ** -0.5
@@ -271,19 +329,36 @@ def mla_sparse_prefill(q: torch.Tensor, kv: torch.Tensor, indices: torch.Tensor,
                        workspace: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Sparse prefill: q bf16 [s_q, h_q, 576], kv bf16 [s_kv, (1,) 576], indices int32 [s_q, (1,) topk]
     -> (out bf16 [s_q, h_q, 512], lse fp32 [h_q, s_q]).  Metadata is computed when not given."""
-    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[-1] != D_QK:
+    _require(q, "q", torch.bfloat16, 3)
+    if q.shape[-1] != D_QK:
         raise ValueError("q must be bf16 [s_q, h_q, 576]")
-    q = q.contiguous()
     s_q, h_q, _ = q.shape
     if kv.dtype != torch.bfloat16 or kv.shape[-1] != D_QK or not kv.is_contiguous():
         raise ValueError("kv must be contiguous bf16 [s_kv, (1,) 576]")
     s_kv = kv.shape[0]
     idx = indices.reshape(s_q, -1) if indices.dim() == 3 else indices
-    if idx.dtype != torch.int32 or idx.dim() != 2 or idx.shape[0] != s_q:
+    _require(idx, "indices", torch.int32, 2)
+    if idx.shape[0] != s_q:
         raise ValueError("indices must be int32 [s_q, (1,) topk]")
-    idx = idx.contiguous()
     topk = idx.shape[1]
-    if tile_md is None or num_splits is None:
+    if (tile_md is None) != (num_splits is None):
+        raise ValueError("pass tile_md and num_splits together (or neither)")
+    if tile_md is not None:
+        _require(tile_md, "tile_md", torch.int32, 2)
+        if tile_md.shape[1] != 8 or tile_md.shape[0] < 1:
+            raise ValueError("tile_md must be int32 [num_sm_parts, 8] from mla_get_metadata_sparse")
+        _require(num_splits, "num_splits", torch.int32, shape=(s_q + 1,))
+    if out is not None:
+        _require(out, "out", torch.bfloat16, shape=(s_q, h_q, D_V))
+    if lse is not None:
+        _require(lse, "lse", torch.float32, shape=(h_q, s_q))
+    if workspace is not None:
+        _require(workspace, "workspace", torch.uint8)
+    if q.is_cuda:
+        q, idx = q.contiguous(), idx.contiguous()
+    _on_device(q.device, q=q, kv=kv, indices=idx, tile_md=tile_md, num_splits=num_splits, out=out, lse=lse,
+               workspace=workspace)
+    if tile_md is None:
         tile_md, num_splits = mla_get_metadata_sparse(1, s_q, topk, h_q, 1, device=q.device, stream=stream)
     num_sm_parts = tile_md.shape[0]
     if out is None:
@@ -303,6 +378,12 @@ def mla_sparse_prefill(q: torch.Tensor, kv: torch.Tensor, indices: torch.Tensor,
 def flash_mla_sparse_fwd(q, kv, indices, sm_scale, d_v=D_V):
     """The spelling of the sparse prefill call on the pages."""
     return mla_sparse_prefill(q, kv, indices, sm_scale, d_v=d_v)
+
+
+def mla_fault_injection_arm(wait_limit_cycles: int, withhold_fill: int = -1) -> None:
+    """Tests only: arm the next mla_decode_kvcache call with a shorter wait bound and a slot fill
+    that its producer skips (see include/mla.h)."""
+    _check(_lib.mla_fault_injection_arm(int(wait_limit_cycles), int(withhold_fill)), "mla_fault_injection_arm")
 
 
 def mla_read_status(workspace: torch.Tensor, reset: bool = False, stream=None) -> int:

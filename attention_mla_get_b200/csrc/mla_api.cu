@@ -1,5 +1,6 @@
 // C-ABI of libmla (declared in include/mla.h): host-side argument checks, workspace
 // partitioning, TMA descriptor encoding and the kernel launches.  No compute happens here.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 
@@ -72,6 +73,10 @@ WorkspaceLayout workspace_layout(int batch, int parts, int rows) {
 }
 
 int rows_per_cta_for(int rows) { return rows <= 16 ? 16 : (rows <= 32 ? 32 : 64); }
+
+// armed by mla_fault_injection_arm, taken (and cleared) by the next mla_decode_kvcache call
+std::atomic<long long> g_fault_wait_limit{0};
+std::atomic<int> g_fault_withhold1{0};
 
 }  // namespace
 
@@ -215,6 +220,8 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   p.row_groups = pair ? (rows + mla::kPairRows - 1) / mla::kPairRows : (rows + rg - 1) / rg;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.wait_limit = g_fault_wait_limit.exchange(0);
+  p.withhold_fill1 = g_fault_withhold1.exchange(0);
 
   mla::OutMaps om;
   if (!encode_out_maps(encode, &om, p.o_part, out, rows, batch, num_sm_parts, rg == 16 ? 16 : 32))
@@ -245,6 +252,10 @@ int mla_get_metadata_sparse(int batch, int s_q, int topk, int h_q, int h_kv, int
   if (!tile_md || !num_splits) return MLA_ERR_NULL_POINTER;
   if (batch < 1 || s_q < 1 || topk < 1 || h_q < 1 || h_q > kMaxRows) return MLA_ERR_BAD_SHAPE;
   if (static_cast<long long>(batch) * s_q >= (1ll << 30)) return MLA_ERR_BAD_SHAPE;
+  // the scheduler's 32-bit prefix sums: total cost = positions * (blocks of topk + 2) < 2^31
+  const long long cost = static_cast<long long>(batch) * s_q *
+                         ((static_cast<long long>(topk) + mla::kBlockTokens - 1) / mla::kBlockTokens + mla::kFixedSplitCost);
+  if (cost >= (1ll << 31)) return MLA_ERR_BAD_SHAPE;
   if (h_kv != 1) return MLA_ERR_BAD_HEADS;
   if (num_sm_parts < 1) return MLA_ERR_BAD_PARTS;
   const int e = mla::launch_scheduler(nullptr, batch * s_q, num_sm_parts, tile_md, num_splits,
@@ -413,6 +424,13 @@ int mla_sparse_prefill(const void* q, const void* kv, int s_kv, const int32_t* i
   cp.vq = s_q;
   e = mla::launch_combine(cp, st);
   return e == 0 ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_fault_injection_arm(long long wait_limit_cycles, int withhold_fill) {
+  if (wait_limit_cycles < 0 || withhold_fill < -1) return MLA_ERR_BAD_SHAPE;
+  g_fault_wait_limit.store(wait_limit_cycles);
+  g_fault_withhold1.store(withhold_fill + 1);
+  return MLA_OK;
 }
 
 int mla_read_status(void* workspace, int reset, int* status, void* stream) {

@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
   const int lane = threadIdx.x & 31;
   const int part = blockIdx.x;
   const int rg = blockIdx.y;  // row group
-  const WaitCtl wc{abort_flag, p.status, kStatusWaitTimeout};
+  const WaitCtl wc{abort_flag, p.status, kStatusWaitTimeout, p.wait_limit > 0 ? p.wait_limit : kWaitLimitCycles};
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMaxSlots; ++i) {
@@ -335,6 +335,8 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
   // launched as a programmatic dependent of the tile scheduler: the set-up above overlapped
   // it; its metadata is complete and visible from here on
   pdl_wait_primary();
+  // metadata the scheduler could not build: its parts are empty, report it
+  if (threadIdx.x == 0 && p.status && p.tile_md[part * kMdInts + 5] != 0) atomicOr(p.status, kStatusBadMetadata);
 
   if (SPARSE && (warp == 4 || warp >= 6)) {
     // ======================= gather producers (token-sparse) =======================
@@ -436,6 +438,12 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       auto fill = [&](int dims0, int natoms, const StepPages& sp, uint64_t pol) -> bool {
         const int s = static_cast<int>(g % C::kNumSlots);
         const uint32_t use = g / C::kNumSlots;
+        if (g + 1 == static_cast<uint32_t>(p.withhold_fill1)) {
+          // fault injection (tests only): this fill is never issued, so its consumer's bounded
+          // wait runs out and the CTA unwinds
+          ++g;
+          return true;
+        }
         if (!mbar_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
         mbar_arrive_expect_tx(bar(kBarSlotFull + s),
                               static_cast<uint32_t>(natoms * (sp.has_b ? 2 : 1) * C::kPageBoxBytes));

@@ -307,6 +307,8 @@ __device__ __forceinline__ uint32_t e4m3x2_times_f16x2(uint32_t codes, uint32_t 
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(scale2));
   return r;
 }
+// Largest scale for which 448 * scale (the largest e4m3 magnitude) is finite in f16.
+constexpr float kF16MaxScale = 65504.0f / 448.0f;
 // The same with the product formed in fp32 (scales outside the f16 normal range).
 __device__ __forceinline__ uint32_t e4m3x2_times_f32(uint32_t codes, float scale) {
   uint32_t h;
@@ -466,6 +468,8 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
   // launched as a programmatic dependent of the tile scheduler: the set-up above overlapped
   // it; its metadata is complete and visible from here on
   pdl_wait_primary();
+  // metadata the scheduler could not build: its parts are empty, report it
+  if (threadIdx.x == 0 && p.status && p.tile_md[part * kMdInts + 5] != 0) atomicOr(p.status, kStatusBadMetadata);
 
   // state the exit sequence needs
   uint32_t fills = 0;  // producer: stage fills issued
@@ -911,12 +915,22 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
     int last_use[kMaxSlots];
     for (int i = 0; i < kMaxSlots; ++i) last_use[i] = -1;
     bool ok = true;
-    // bf16 -> f16 in place over `bytes` of shared memory at `base`
-    auto to_f16 = [&](uint32_t base, int bytes) {
+    // largest |bf16| bit pattern seen by to_f16 in each 16-bit half, and whether a scale let
+    // code * scale leave the f16 range: reported as a status bit at the end
+    uint32_t mag = 0;
+    bool scale_range = false;
+    // bf16 -> f16 in place over `bytes` of shared memory at `base`; the magnitudes of the first
+    // `checked` 16-byte chunks enter the range check (RoPE slots: the rows of tokens that exist,
+    // 8 chunks per token row; page tails hold undefined data that never reaches a result)
+    auto to_f16 = [&](uint32_t base, int bytes, int checked) {
       for (int c = dt; c < bytes / 16; c += kDequantThreads) {
         uint32_t w0, w1, w2, w3;
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
                      : "r"(base + 16u * c));
+        if (c < checked) {
+          mag = __vmaxu2(mag, __vmaxu2(w0 & 0x7FFF7FFFu, w1 & 0x7FFF7FFFu));
+          mag = __vmaxu2(mag, __vmaxu2(w2 & 0x7FFF7FFFu, w3 & 0x7FFF7FFFu));
+        }
         st_shared_v4(base + 16u * c, bf16x2_to_f16x2(w0), bf16x2_to_f16x2(w1), bf16x2_to_f16x2(w2),
                      bf16x2_to_f16x2(w3));
       }
@@ -946,6 +960,9 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
           float scale;
           asm volatile("ld.shared.f32 %0, [%1];" : "=f"(scale)
                        : "r"(raw + kRawCodeBytes + pg * (kRawScaleBytes / 2) + i * 16u + 4u * grp));
+          // 448 * scale must stay within f16 (a quantiser's scale is max|x| / 448, so this is
+          // exactly the condition that the largest value of the group fits)
+          scale_range |= !(scale <= kF16MaxScale);
           dequant_row(raw + pg * (kRawCodeBytes / 2) + i * 128u, dst, hstride, i, scale);
         } else {
           // tokens outside the request or the chunk: zeros (masked in S^T, 0 rows of V)
@@ -973,7 +990,7 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
       const int L = p.cache_seqlens[b];
       const int n = (c1 - c0 + 1) / 2;
       ok &= warp_pwait(bar(kBarQFull), qc & 1u, wc, lane);
-      if (ok) to_f16(sQ, kQBytes);
+      if (ok) to_f16(sQ, kQBytes, kQBytes / 16);
       ++qc;
       if (!publish(kBarQReady)) break;
       for (int e = 0; ok && e < 2 * n; ++e) {
@@ -982,7 +999,12 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
         order_at(e, n, is_v, t);
         if (!is_v) {
           ok &= warp_pwait(bar(kBarRopeFull), rc & 1u, wc, lane);
-          if (ok) to_f16(sRope, kRopeBytes);
+          if (ok) {
+            // this CTA's block of the step: its tokens below the chunk end and the request length
+            const int tb = c0 + 2 * t + static_cast<int>(rank);
+            const int valid = tb < c1 ? min(kBlockTokens, max(0, L - tb * kBlockTokens)) : 0;
+            to_f16(sRope, kRopeBytes, valid * 8);
+          }
           ++rc;
           if (!publish(kBarRopeReady)) { ok = false; break; }
           // K(t) stage j: dims 128j.. of this CTA's block; [dim half][page][64 tokens][64 dims]
@@ -999,6 +1021,9 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
       // the last pair commits on this CTA's stage barriers have landed before it may exit
       for (int s = 0; s < kNumSlots; ++s)
         if (last_use[s] >= 0) drain_wait(bar(kBarSlotEmpty + s), static_cast<uint32_t>(last_use[s]) & 1u);
+    // a bf16 value of q or of a RoPE dim of magnitude >= 65536 (0x4780) is infinite in f16
+    const bool range_bad = scale_range || (mag & 0xFFFFu) >= 0x4780u || (mag >> 16) >= 0x4780u;
+    if (__any_sync(0xffffffffu, range_bad) && lane == 0 && p.status) atomicOr(p.status, kStatusF16Range);
     __syncwarp();
     }
   } else {

@@ -20,6 +20,11 @@ constexpr int kFp8TokenBytes = 656;
 
 // device status bits (sticky, in the first word of the workspace)
 constexpr int kStatusWaitTimeout = 1;
+constexpr int kStatusBadMetadata = 2;  // the tile scheduler flagged its metadata (see kMdOverflow)
+constexpr int kStatusF16Range = 4;     // FP8 CTA pair: an operand left the f16 range
+// tile_md[part][5]: nonzero when the scheduler could not build the metadata (the total cost of
+// the batch does not fit its 32-bit prefix sums); every part is then empty
+constexpr int kMdOverflow = 1;
 
 struct DecodeParams {
   const int32_t* block_table;
@@ -47,6 +52,10 @@ struct DecodeParams {
   int topk;
   int vq;
   int kv_len;             // sparse prefill: tokens of the one contiguous cache (cache_seqlens null)
+  // fault injection for tests of the bounded waits (mla_fault_injection_arm; single-CTA bf16
+  // kernel only): a shorter wait bound, and 1 + the index of a slot fill the producer skips
+  long long wait_limit;   // 0: the default bound
+  int withhold_fill1;     // 0: none
 };
 
 struct CombineParams {

@@ -16,7 +16,12 @@
 //   - every call on a device shares the one array and leaves its contents behind; the device
 //     status word is cleared (cudaMemsetAsync, no allocation) at the start of each call, the
 //     partial results are always written before they are read;
-//   - calls that overlap on the GPU (other streams, or other host threads) race on the array.
+//   - calls that overlap on the GPU (other streams, or other host threads) race on the array;
+//   - mla_noalloc_read_status reads the status word back (the caller has no workspace pointer
+//     to hand to mla_read_status);
+//   - the cached address belongs to the device's current context: after cudaDeviceReset the
+//     module is loaded again and the array may move, so do not call these entry points after
+//     resetting a device in the same process.
 // Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 #include <mutex>
 
@@ -75,6 +80,20 @@ int mla_decode_kvcache_noalloc(const void* q, const void* kvcache, int64_t num_b
   return mla_decode_kvcache(q, kvcache, num_blocks, block_table, max_blocks, cache_seqlens, batch, s_q, h_q, h_kv,
                             d_v, tile_md, num_sm_parts, num_splits, softmax_scale, causal, kv_dtype, out, lse, ws,
                             kNoAllocScratchBytes, stream);
+}
+
+int mla_noalloc_read_status(int reset, int* status, void* stream) {
+  if (!status) return MLA_ERR_NULL_POINTER;
+  void* ws = nullptr;
+  const int e = scratch_for_current_device(&ws);
+  if (e != MLA_OK) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  *status = v;
+  if (reset && cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
 }
 
 }  // extern "C"

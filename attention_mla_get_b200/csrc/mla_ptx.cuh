@@ -61,6 +61,7 @@ struct WaitCtl {
   volatile int* abort_flag;   // shared memory
   int* status;                // global memory (may be null)
   int code;
+  long long limit;            // cycles (kWaitLimitCycles unless a test asks for less)
 };
 
 static __device__ __noinline__ void signal_timeout(const WaitCtl& c) {
@@ -75,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*c.abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > c.limit) {
       signal_timeout(c);
       return false;
     }

@@ -14,7 +14,8 @@
 //   num_splits = prefix sum of chunks; first_split = num_splits[begin_b] + p - floor((C_b+F)/q)
 // Every quantity is a closed form of prefix sums, so one CTA of 1024 threads computes the
 // metadata in a few microseconds: a scan of costs, a binary search per part, a scan of
-// chunk counts.
+// chunk counts.  A batch whose total cost T does not fit in 31 bits gets empty parts flagged
+// with kMdOverflow in column 5 (and no splits); the decode kernels report it as a status bit.
 #include "mla_internal.h"
 #include "mla_ptx.cuh"
 
@@ -90,6 +91,22 @@ __global__ void __launch_bounds__(kSchedThreads)
   const long long T = carry;
   const long long q = T > 0 ? (T + parts - 1) / parts : 1;
   __syncthreads();
+  if (T > 0x7fffffffll) {
+    // the prefix sums above were stored as 32-bit values and wrapped: publish empty parts
+    // flagged kMdOverflow (the decode kernels raise a status bit) and no splits at all
+    for (int p = tid; p < parts; p += nthreads) {
+      int32_t* row = md + static_cast<long long>(p) * kMdInts;
+      row[0] = batch;
+      row[1] = 0;
+      row[2] = batch;
+      row[3] = 0;
+      row[4] = 0;
+      row[5] = kMdOverflow;
+      row[6] = row[7] = 0;
+    }
+    for (int b = tid; b <= batch; b += nthreads) ns[b] = 0;
+    return;
+  }
 
   // pass 2: per part, the first block at a position >= x (binary search on C_{b+1})
   const int32_t* cum = on_chip ? s_cum : ns;  // C_{b+1} at index b + 1

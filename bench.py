@@ -19,8 +19,14 @@ e2e       the same metric when every step also copies its inputs (q, block_table
           read back (two copy streams, double-buffered device staging) while step k computes;
           sparse prefill, which has no session call, runs the same pipeline from Python.  The
           timed region runs from before the first copy-in to after the last read-back.
-roofline  the decode call (main kernel + combine), algorithmic bytes per launch divided by
-          its mean CUDA-event duration, against the measured HBM copy bandwidth.
+roofline  the decode call (main kernel + combine): algorithmic bytes (or FLOPs) per call divided by
+          its mean duration, timed in a loop of decode calls alone (CUDA events at the ends
+          of the loop), against the measured HBM copy bandwidth or cuBLAS bf16 rate, with the
+          fraction of the nominal B200 figures (8 TB/s, 2.25 PFLOP/s) beside it.  The whole-step
+          loop that gives `value` records events only before its first and after its last
+          step, so the scheduler -> decode programmatic launch chain runs undisturbed.
+per_workload  the same figures for the other workloads (variable-length h128, causal s_q 2,
+          FP8 cache, token-sparse decode, sparse prefill), a few steps each, on a 1-GPU run.
 cpu_baseline  the fp64 oracle timed on this host's cores on a bounded sample of requests.
 
 With N > 1 (torchrun), every rank runs its own batch of requests on its own GPU (requests
@@ -51,8 +57,8 @@ def _peaks():
 
 
 class ClockSampler:
-    """Samples SM clock, power and clock-event reasons through NVML every 10 ms while the
-    timed region runs (nvidia-smi as a fallback)."""
+    """Samples SM clock, power and clock-event reasons through NVML every 2 ms while the
+    timed region runs."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown"}
 
@@ -90,7 +96,7 @@ class ClockSampler:
                 self.samples.append((time.perf_counter(), *self._read()))
             except Exception:
                 pass
-            self._stop.wait(0.01)
+            self._stop.wait(0.002)
 
     def __enter__(self):
         if self._h is not None:
@@ -206,18 +212,156 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+class DeviceRun:
+    """One workload's inputs resident on the device and the calls of one step: the tile
+    scheduler (mla_get_metadata) and the decode call (main kernel + combine)."""
+
+    def __init__(self, case, dev, mla):
+        import torch
+        import mla_inputs as mi
+        self.case, self.dev, self.mla = case, dev, mla
+        self.q = torch.from_numpy(case.q_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        if case.kv_format == "bf16":
+            self.kv = torch.from_numpy(case.kv.view(np.int16)).view(torch.bfloat16).reshape(
+                case.num_blocks, mi.PAGE, 1, mi.D_QK).to(dev)
+        else:
+            self.kv = torch.from_numpy(case.kv).to(dev)
+        self.bt = torch.from_numpy(case.block_table).to(dev)
+        self.sl = torch.from_numpy(case.cache_seqlens).to(dev)
+        self.sparse = case.indices is not None
+        self.idx = torch.from_numpy(case.indices).to(dev) if self.sparse else None
+        R = case.rows
+        # token-sparse: the scheduler's requests are the batch * s_q query positions of h_q rows
+        self.parts = mla.mla_num_sm_parts(case.h_q if self.sparse else R, 1, dev.index)
+        self.ws = torch.zeros(mla.mla_workspace_size(case.batch * case.s_q, self.parts, case.h_q, 1) if self.sparse
+                              else mla.mla_workspace_size(case.batch, self.parts, R, 1), dtype=torch.uint8, device=dev)
+        self.out = torch.empty((case.batch, case.s_q, case.h_q, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((case.batch, case.h_q, case.s_q), dtype=torch.float32, device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.prefill = bool(case.meta.get("prefill"))
+        if self.prefill:
+            s_kv = int(case.cache_seqlens[0])
+            self.kv = self.kv.reshape(-1, mi.D_QK)[:s_kv].reshape(s_kv, 1, mi.D_QK).contiguous()
+            self.q = self.q[0].contiguous()
+            self.idx = self.idx[0].contiguous()
+            self.out = self.out[0]
+            self.lse = self.lse[0]
+
+    def metadata(self, sl_):
+        c, mla = self.case, self.mla
+        if self.sparse:
+            return mla.mla_get_metadata_sparse(c.batch, c.s_q, c.topk, c.h_q, 1, num_sm_parts=self.parts,
+                                               device=self.dev)
+        return mla.mla_get_metadata(sl_, c.rows, 1, num_sm_parts=self.parts)
+
+    def decode_into(self, q_, bt_, sl_, idx_, md, ns, out_, lse_):
+        c, mla = self.case, self.mla
+        if self.prefill:
+            mla.mla_sparse_prefill(q_, self.kv, idx_, c.softmax_scale, tile_md=md, num_splits=ns, out=out_, lse=lse_,
+                                   workspace=self.ws)
+        elif self.sparse:
+            mla.mla_decode_kvcache_sparse(q_, self.kv, bt_, sl_, idx_, 512, md, ns, softmax_scale=c.softmax_scale,
+                                          out=out_, lse=lse_, workspace=self.ws)
+        else:
+            mla.mla_decode_kvcache(q_, self.kv, bt_, sl_, 512, md, ns, softmax_scale=c.softmax_scale,
+                                   causal=c.causal, out=out_, lse=lse_, workspace=self.ws)
+
+    def step(self):
+        md, ns = self.metadata(self.sl)
+        self.decode_into(self.q, self.bt, self.sl, self.idx, md, ns, self.out, self.lse)
+
+    def measure(self, steps, warmup, barrier, reduce_max):
+        """Device time of `steps` whole steps (events only at the ends of the loop: the decode
+        kernel is a programmatic dependent of the scheduler, and an event between them would
+        serialise the pair), then, in a separate loop, of `steps` decode calls alone on fixed
+        metadata (the roofline's kernel time).  Both are max-over-ranks."""
+        import torch
+        for _ in range(warmup):
+            self.step()
+        barrier()
+        # clocks under the same load for ~0.3 s just before the timed region (a short timed
+        # region holds only a few samples); reported beside the timed region's own samples
+        with ClockSampler(self.dev) as soak:
+            t0 = time.perf_counter()
+            while time.perf_counter() - t0 < 0.3:
+                for _ in range(max(1, steps)):
+                    self.step()
+                torch.cuda.synchronize(self.dev)
+            soak.mark(t0, time.perf_counter())
+        barrier()
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(self.dev) as clk:
+            t_wall0 = time.perf_counter()
+            start.record(self.stream)
+            for _ in range(steps):
+                self.step()
+            stop.record(self.stream)
+            barrier()
+            clk.mark(t_wall0, time.perf_counter())
+        ms_total = reduce_max(start.elapsed_time(stop))
+        # decode calls alone (metadata computed once, outside the loop)
+        md, ns = self.metadata(self.sl)
+        for _ in range(2):
+            self.decode_into(self.q, self.bt, self.sl, self.idx, md, ns, self.out, self.lse)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(self.stream)
+        for _ in range(steps):
+            self.decode_into(self.q, self.bt, self.sl, self.idx, md, ns, self.out, self.lse)
+        b.record(self.stream)
+        barrier()
+        decode_ms = reduce_max(a.elapsed_time(b)) / steps
+        status = self.mla.mla_read_status(self.ws)
+        clocks = clk.summary()
+        clocks["soak"] = soak.summary()
+        return {"ms_total": ms_total, "decode_ms": decode_ms, "clocks": clocks, "status": status}
+
+
+def roofline_of(units, decode_ms, ms_step, peaks):
+    """Roofline figures of one workload: the bound is the slower of its bytes at HBM peak and
+    its FLOPs at tensor peak (measured peaks), `achieved` is the decode call's rate, and the
+    same fraction is also given against the nominal B200 figures (8 TB/s, 2.25 PFLOP/s dense
+    bf16) and, for tensor-bound work, against the sustained cuBLAS figure."""
+    hbm_peak, tc_peak, tc_sustained, peak_kind = peaks
+    hbm_bound = units["bytes"] / (hbm_peak * 1e9) >= units["flops"] / (tc_peak * 1e12)
+    gbs = units["bytes"] / (decode_ms * 1e-3) / 1e9
+    tfs = units["flops"] / (decode_ms * 1e-3) / 1e12
+    if hbm_bound:
+        r = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+             "peak_kind": peak_kind + " copy bandwidth", "nominal_peak": NOMINAL_HBM_GBS,
+             "frac_nominal": gbs / NOMINAL_HBM_GBS}
+    else:
+        r = {"bound": "tensor", "achieved": tfs, "peak": tc_peak, "unit": "TFLOP/s", "frac": tfs / tc_peak,
+             "peak_kind": peak_kind + " cuBLAS bf16 burst", "frac_sustained": tfs / tc_sustained,
+             "sustained_peak": tc_sustained, "nominal_peak": NOMINAL_BF16_TFLOPS,
+             "frac_nominal": tfs / NOMINAL_BF16_TFLOPS}
+    roof_time = max(units["bytes"] / (hbm_peak * 1e9), units["flops"] / (tc_peak * 1e12))
+    r["step_frac"] = roof_time / (ms_step * 1e-3)
+    return r
+
+
+DEFAULT_WORKLOAD = "mem_b128_h16_L8192"
+PER_WORKLOADS = ("varlen_b128_h128", "causal_b64_sq2_h128", "fp8_b128_h128_L16384",
+                 "sparse_b128_h128_L8192_topk2048", "sparse_prefill_s4096_h128_kv8192_topk2048")
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="mem_b128_h16_L8192")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="run the first BATCH requests of the workload (profiling captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="time only the headline workload (by default a 1-GPU run also times the other workloads)")
+    ap.add_argument("--per-steps", type=int, default=20, help="timed steps of each other workload")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -228,7 +372,7 @@ def main():
     import mla_inputs as mi
     w = mi.WORKLOADS[args.workload]
     metric = "MLA paged-KV decode TFLOP/s and KV HBM GB/s; fraction of B200 roofline"
-    hbm_peak, tc_peak, tc_sustained, peak_kind = _peaks()
+    peaks = _peaks()
 
     if args.impl == "reference":
         # the reference arm is the fp64 oracle on host cores (rank 0 only)
@@ -263,92 +407,21 @@ def main():
     dev = torch.device("cuda", local)
     import attention_mla_get_b200 as mla
 
-    def to_device(c, device):
-        qd = torch.from_numpy(c.q_bits.view(np.int16)).view(torch.bfloat16).to(device)
-        if c.kv_format == "bf16":
-            kvd = torch.from_numpy(c.kv.view(np.int16)).view(torch.bfloat16).reshape(
-                c.num_blocks, mi.PAGE, 1, mi.D_QK).to(device)
-        else:
-            kvd = torch.from_numpy(c.kv).to(device)
-        return qd, kvd, torch.from_numpy(c.block_table).to(device), torch.from_numpy(c.cache_seqlens).to(device)
-
-    # every rank owns its own requests (seed shifted by rank): independent problems
-    case = rank_case(args.workload, rank, args.batch)
-    units = mi.workload_units(case)
-    q, kv, bt, sl = to_device(case, dev)
-    sparse = case.indices is not None
-    idx = torch.from_numpy(case.indices).to(dev) if sparse else None
-    R = case.rows
-    # token-sparse: the scheduler's requests are the batch * s_q query positions of h_q rows
-    parts = mla.mla_num_sm_parts(case.h_q if sparse else R, 1, local)
-    ws = torch.zeros(mla.mla_workspace_size(case.batch * case.s_q, parts, case.h_q, 1) if sparse else
-                     mla.mla_workspace_size(case.batch, parts, R, 1), dtype=torch.uint8, device=dev)
-    out = torch.empty((case.batch, case.s_q, case.h_q, 512), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((case.batch, case.h_q, case.s_q), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    prefill = bool(case.meta.get("prefill"))
-    if prefill:
-        s_kv = int(case.cache_seqlens[0])
-        kv = kv.reshape(-1, mi.D_QK)[:s_kv].reshape(s_kv, 1, mi.D_QK).contiguous()
-        q = q[0].contiguous()
-        idx = idx[0].contiguous()
-        out = out[0]
-        lse = lse[0]
-
-    def metadata(sl_):
-        if sparse:
-            return mla.mla_get_metadata_sparse(case.batch, case.s_q, case.topk, case.h_q, 1, num_sm_parts=parts,
-                                               device=dev)
-        return mla.mla_get_metadata(sl_, R, 1, num_sm_parts=parts)
-
-    def decode_into(q_, bt_, sl_, idx_, md, ns, out_, lse_):
-        if prefill:
-            mla.mla_sparse_prefill(q_, kv, idx_, case.softmax_scale, tile_md=md, num_splits=ns, out=out_, lse=lse_,
-                                   workspace=ws)
-        elif sparse:
-            mla.mla_decode_kvcache_sparse(q_, kv, bt_, sl_, idx_, 512, md, ns, softmax_scale=case.softmax_scale,
-                                          out=out_, lse=lse_, workspace=ws)
-        else:
-            mla.mla_decode_kvcache(q_, kv, bt_, sl_, 512, md, ns, softmax_scale=case.softmax_scale,
-                                   causal=case.causal, out=out_, lse=lse_, workspace=ws)
-
-    def decode(q_, bt_, sl_, idx_, md, ns):
-        decode_into(q_, bt_, sl_, idx_, md, ns, out, lse)
-
-    def step():
-        md, ns = metadata(sl)
-        decode(q, bt, sl, idx, md, ns)
-
     def barrier():
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    for _ in range(args.warmup):
-        step()
-    barrier()
-
-    # ---- device-timed steps, with per-call events for the decode kernel's roofline ----
-    md0, ns0 = metadata(sl)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    with ClockSampler(dev) as clk:
-        t_wall0 = time.perf_counter()
-        start.record(stream)
-        for i in range(args.steps):
-            md, ns = metadata(sl)
-            ev[i][0].record(stream)
-            decode(q, bt, sl, idx, md, ns)
-            ev[i][1].record(stream)
-        stop.record(stream)
-        barrier()
-        clk.mark(t_wall0, time.perf_counter())
-    ms_total = max_over_ranks(start.elapsed_time(stop), world, dev)
-    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
-    status = mla.mla_read_status(ws)
+    # every rank owns its own requests (seed shifted by rank): independent problems
+    case = rank_case(args.workload, rank, args.batch)
+    units = mi.workload_units(case)
+    run = DeviceRun(case, dev, mla)
+    m = run.measure(args.steps, args.warmup, barrier, lambda x: max_over_ranks(x, world, dev))
+    ms_total, decode_ms, clk, status = m["ms_total"], m["decode_ms"], m["clocks"], m["status"]
+    q, kv, bt, sl, idx, out, lse = run.q, run.kv, run.bt, run.sl, run.idx, run.out, run.lse
+    sparse, prefill, parts, stream = run.sparse, run.prefill, run.parts, run.stream
+    metadata, decode_into = run.metadata, run.decode_into
 
     # ---- end to end through the C-ABI with host buffers ----
     q_h = q.cpu().pin_memory()
@@ -420,6 +493,32 @@ def main():
     if session is not None:
         session.close()
 
+    # ---- the other workloads (one GPU: rank 0 of a 1-rank job only), a few steps each ----
+    per_workload = None
+    if world == 1 and not args.no_per_workload and args.batch is None and args.workload == DEFAULT_WORKLOAD:
+        per_workload = {}
+        del run, q, kv, bt, sl, idx, out, lse, bufs, metadata, decode_into
+        torch.cuda.empty_cache()
+        for name in PER_WORKLOADS:
+            wcase = mi.make_workload(name, poison=False)
+            wunits = mi.workload_units(wcase)
+            wrun = DeviceRun(wcase, dev, mla)
+            wm = wrun.measure(args.per_steps, 3, barrier, lambda x: x)
+            ms_step = wm["ms_total"] / args.per_steps
+            per_workload[name] = {
+                "ms_per_step": ms_step, "decode_ms": wm["decode_ms"],
+                "gbs": wunits["bytes"] / (ms_step * 1e-3) / 1e9, "tflops": wunits["flops"] / (ms_step * 1e-3) / 1e12,
+                "steps": args.per_steps, "warmup": 3,
+                "roofline": roofline_of(wunits, wm["decode_ms"], ms_step, peaks),
+                "clocks": wm["clocks"], "device_status": wm["status"],
+                "gpu_launches": 3 * args.per_steps,
+                "config": {"batch": wcase.batch, "s_q": wcase.s_q, "h_q": wcase.h_q, "causal": wcase.causal,
+                           "kv": wcase.kv_format, "topk": wcase.topk, "seqlens": mi.WORKLOADS[name].seqlens,
+                           "kv_bytes": wunits["kv_bytes"], "flops": wunits["flops"]},
+            }
+            del wrun
+            torch.cuda.empty_cache()
+
     if rank != 0:
         if world > 1:
             dist.barrier()
@@ -429,12 +528,9 @@ def main():
     total_bytes = units["bytes"] * world * args.steps
     value = total_bytes / (ms_total * 1e-3) / 1e9
     tflops = units["flops"] * world * args.steps / (ms_total * 1e-3) / 1e12
-    hbm_bound = units["bytes"] / (hbm_peak * 1e9) >= units["flops"] / (tc_peak * 1e12)
-    if hbm_bound:
-        achieved, peak, runit = units["bytes"] / (decode_ms * 1e-3) / 1e9, hbm_peak, "GB/s"
-    else:
-        achieved, peak, runit = units["flops"] / (decode_ms * 1e-3) / 1e12, tc_peak, "TFLOP/s"
-    roof_time = max(units["bytes"] / (hbm_peak * 1e9), units["flops"] / (tc_peak * 1e12))
+    roof = roofline_of(units, decode_ms, ms_total / args.steps, peaks)
+    roof["kernel"] = "mla_decode_kvcache (split-KV main + combine), decode calls alone"
+    roof["traffic"] = TRAFFIC.get(args.workload) if roof["bound"] == "hbm" else None
     line = {
         "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
@@ -447,18 +543,18 @@ def main():
                    "kv": case.kv_format, "kv_bytes": units["kv_bytes"], "l2": "inputs larger than L2 (no flush)",
                    "parallelism": f"replicas x{world} (independent requests per GPU)"},
         "tflops": tflops,
-        "roofline_fraction": roof_time / (ms_total / args.steps * 1e-3),
-        "roofline": {"bound": "hbm" if hbm_bound else "tensor",
-                     "kernel": "mla_decode_kvcache (split-KV main + combine)", "achieved": achieved,
-                     "peak": peak, "unit": runit, "frac": achieved / peak, "traffic": TRAFFIC.get(args.workload),
-                     "peak_kind": peak_kind + (" copy bandwidth" if hbm_bound else " cuBLAS bf16 burst")},
+        "roofline_fraction": roof["step_frac"],
+        "roofline": roof,
+        "decode_ms": decode_ms,
         "e2e": None if e2e_ms is None else {
             "value": units["bytes"] * world * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clk,
         "device_status": status,
     }
+    if per_workload is not None:
+        line["per_workload"] = per_workload
     if not args.no_cpu_baseline:
         r = oracle_baseline(case, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": r["units"]["bytes"] / r["seconds"] / 1e9, "unit": "GB/s",

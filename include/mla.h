@@ -70,11 +70,20 @@ extern "C" {
 /* Device status bits written into the workspace by the kernels (sticky until reset). */
 #define MLA_STATUS_WAIT_TIMEOUT 1     /* an internal pipeline wait ran past its bound (~1 s);
                                          the outputs of that call are undefined */
+#define MLA_STATUS_BAD_METADATA 2     /* the tile metadata passed in was flagged by the scheduler
+                                         as unbuildable (see mla_get_metadata); the call wrote
+                                         O = 0 and LSE = -inf for every row */
+#define MLA_STATUS_F16_RANGE 4        /* FP8 cache with more than 64 query rows per request (f16
+                                         tensor-core operands): a value of q or of a RoPE dim of
+                                         magnitude >= 65536, or a scale above 65504 / 448, left
+                                         the f16 range; that call's outputs are unreliable */
 
 /*
- * Number of scheduler parts ("SM parts") for a problem: the number of CTAs that share one
- * chunk of pages is G = ceil(rows_per_kv_head / 64) (1 when rows <= 64), so
- * num_sm_parts = max(1, SM count of `device` / (h_kv * G)).
+ * Number of scheduler parts ("SM parts") for a problem.  A chunk of pages is processed by
+ * G SMs: G = 1 when rows_per_kv_head <= 64 (one CTA carries up to 64 query rows), otherwise
+ * G = 2 * ceil(rows_per_kv_head / 128) (a pair of CTAs on the two SMs of a TPC carries 128
+ * rows), so num_sm_parts = max(1, SM count of `device` / (h_kv * G)).  For example, on 148
+ * SMs: 148 parts for 16 rows, 74 for 128, 37 for 192 or 256.
  *   rows_per_kv_head  s_q * h_q / h_kv
  * Returns the count (>= 1) or a negative MLA_ERR_* code.
  */
@@ -89,6 +98,10 @@ MLA_API int mla_num_sm_parts(int rows_per_kv_head, int h_kv, int device);
  *   tile_md        device int32 [num_sm_parts, 8] (written): per part
  *                  {begin_b, begin_block, end_b, end_block, first_split, 0, 0, 0}
  *   num_splits     device int32 [batch + 1] (written): prefix count of chunks per request
+ * The total cost (sum over requests with tokens of ceil(L_b / 128) + 2) must stay below 2^31.
+ * The lengths are device data, so this is checked on the device: a batch above it gets every
+ * part empty with tile_md[p][5] = 1 and num_splits all 0, and a decode call given that
+ * metadata raises MLA_STATUS_BAD_METADATA in its workspace status word.
  * Errors: MLA_ERR_NULL_POINTER, MLA_ERR_BAD_SHAPE (batch < 1), MLA_ERR_BAD_HEADS,
  *         MLA_ERR_BAD_PARTS, MLA_ERR_CUDA.
  */
@@ -116,8 +129,10 @@ MLA_API size_t mla_workspace_size(int batch, int num_sm_parts, int rows_per_kv_h
  *   causal         0 / 1
  *   kv_dtype       MLA_KV_BF16 or MLA_KV_FP8.  With MLA_KV_FP8 and more than 64 query rows per
  *                  request the products run on f16 tensor cores: q, the RoPE dims and every
- *                  code * scale must stay within the f16 range (|x| < 65504; scales up to 146);
- *                  e4m3 NaN codes are not expected (a quantised cache holds none)
+ *                  code * scale must stay within the f16 range (|x| < 65504; scales up to
+ *                  65504 / 448 = 146.2); a call that meets a value outside it raises
+ *                  MLA_STATUS_F16_RANGE.  e4m3 NaN codes are not expected (a quantised cache
+ *                  holds none)
  *   out            device bf16 [batch, s_q, h_q, 512] (written)
  *   lse            device fp32 [batch, h_q, s_q] (written)
  *   workspace      device scratch of >= mla_workspace_size(batch, num_sm_parts, s_q*h_q, h_kv) bytes,
@@ -153,6 +168,17 @@ MLA_API int mla_decode_kvcache_noalloc(const void* q, const void* kvcache, int64
                                        int kv_dtype, void* out, float* lse, void* stream);
 
 /*
+ * Device status word (MLA_STATUS_* bits) of the last mla_decode_kvcache_noalloc call on the
+ * current device, which lives in that call's built-in array (callers of the no-alloc call have
+ * no workspace of their own to read it from).  Waits on `stream` (enqueue it on the stream of
+ * the decode call), copies the word into *status and, when `reset` is nonzero, clears it.
+ * Like the decode call it allocates nothing; it shares the array with it, so read the status
+ * before the next no-alloc call on the device clears it.  Errors: MLA_ERR_NULL_POINTER,
+ * MLA_ERR_NO_DEVICE, MLA_ERR_CUDA.  (The FlashMLA pages have no counterpart of this call.)
+ */
+MLA_API int mla_noalloc_read_status(int reset, int* status, void* stream);
+
+/*
  * Token-sparse decode (the `topk` argument of get_mla_metadata and the `indices` argument of
  * flash_mla_with_kvcache on the gitcode FlashMLA page, "解码阶段使用示例" / "稀疏解码场景").
  * The page names the arguments but not their shape; this library's reading:
@@ -165,7 +191,9 @@ MLA_API int mla_decode_kvcache_noalloc(const void* q, const void* kvcache, int64
  * Every query position is scheduled as a request of topk tokens:
  *   mla_get_metadata_sparse  tile_md [num_sm_parts, 8] and num_splits [batch * s_q + 1] for
  *                            batch * s_q positions of topk tokens; num_sm_parts from
- *                            mla_num_sm_parts(h_q, h_kv)
+ *                            mla_num_sm_parts(h_q, h_kv).  MLA_ERR_BAD_SHAPE when
+ *                            batch * s_q * (ceil(topk / 128) + 2) >= 2^31 (the scheduler's
+ *                            cost sums are 32-bit)
  *   mla_decode_kvcache_sparse  as mla_decode_kvcache (bf16 cache only: MLA_ERR_BAD_KV_DTYPE
  *                            otherwise), with the workspace of
  *                            mla_workspace_size(batch * s_q, num_sm_parts, h_q, h_kv) bytes
@@ -243,6 +271,23 @@ MLA_API int mla_session_join(mla_session* session, void* stream);
 MLA_API int mla_session_status(mla_session* session, int reset, int* status);
 
 MLA_API int mla_session_destroy(mla_session* session);
+
+/*
+ * Fault injection for tests of the kernels' bounded waits (the pages have no counterpart; it
+ * exists so that the time-out path can be exercised without faulting or hanging a GPU).  Arms
+ * the next mla_decode_kvcache call made in this process, which then uses
+ *   wait_limit_cycles  as the bound of every pipeline wait, in SM clock cycles (0: the default
+ *                      bound of about one second), and
+ *   withhold_fill      the index of a shared-memory slot fill (counted from 0 over the call's
+ *                      CTA) that the copy producer skips (-1: none).  The slot's consumer then
+ *                      waits in vain until the bound runs out, sets MLA_STATUS_WAIT_TIMEOUT,
+ *                      and every role of the CTA unwinds (copies in flight are drained, tensor
+ *                      memory is freed); the call's outputs are undefined.
+ * Only the single-CTA bf16 kernel (up to 64 query rows per request) honours the setting; the
+ * next call takes and clears it whichever kernel it runs.  Errors: MLA_ERR_BAD_SHAPE for a
+ * negative limit or a fill index below -1.
+ */
+MLA_API int mla_fault_injection_arm(long long wait_limit_cycles, int withhold_fill);
 
 /*
  * Reads the device status word of a workspace into *status (host pointer).  This call

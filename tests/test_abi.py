@@ -38,10 +38,10 @@ def _declared():
 def test_every_declared_symbol_is_exported(lib):
     names = _declared()
     assert set(names) == {"mla_num_sm_parts", "mla_get_metadata", "mla_workspace_size", "mla_decode_kvcache",
-                          "mla_decode_kvcache_noalloc", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
+                          "mla_decode_kvcache_noalloc", "mla_noalloc_read_status", "mla_get_metadata_sparse", "mla_decode_kvcache_sparse",
                           "mla_sparse_prefill", "mla_session_create", "mla_session_decode", "mla_session_join",
                           "mla_session_status", "mla_session_destroy",
-                          "mla_read_status", "mla_strerror", "mla_version"}
+                          "mla_read_status", "mla_fault_injection_arm", "mla_strerror", "mla_version"}
     so = os.path.join(ROOT, "attention_mla_get_b200", "libmla.so")
     nm = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True).stdout
     exported = set(re.findall(r" T (mla_\w+)", nm))
@@ -61,6 +61,20 @@ def test_built_for_sm100a():
     # the embedded fatbin names its target architecture
     data = open(so, "rb").read()
     assert b"sm_100a" in data
+
+
+def test_noalloc_read_status_rejects_null(lib):
+    lib.mla_noalloc_read_status.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    lib.mla_noalloc_read_status.restype = ctypes.c_int
+    assert lib.mla_noalloc_read_status(0, None, None) == -1
+
+
+def test_fault_injection_arm_argument_errors(lib):
+    lib.mla_fault_injection_arm.argtypes = [ctypes.c_longlong, ctypes.c_int]
+    lib.mla_fault_injection_arm.restype = ctypes.c_int
+    assert lib.mla_fault_injection_arm(-1, -1) == -7
+    assert lib.mla_fault_injection_arm(100, -2) == -7
+    assert lib.mla_fault_injection_arm(0, -1) == 0   # disarmed: the default bound, no withheld fill
 
 
 def test_strerror_and_version(lib):
@@ -145,6 +159,9 @@ def test_sparse_argument_errors_are_reported_before_any_launch(lib):
     assert g(2, 1, 0, 16, 1, fake, 4, fake, None) == -7
     assert g(2, 1, 64, 16, 2, fake, 4, fake, None) == -4
     assert g(2, 1, 64, 16, 1, fake, 0, fake, None) == -8
+    # the scheduler's cost sums are 32-bit: batch * s_q * (ceil(topk / 128) + 2) must stay below 2^31
+    assert g(1 << 29, 1, 256, 16, 1, fake, 4, fake, None) == -7       # 2^29 * 4 = 2^31
+    assert g(1 << 20, 1, 128 * 2046, 16, 1, fake, 4, fake, None) == -7  # 2^20 * 2048 = 2^31
 
 
 def test_session_argument_errors(lib):

@@ -39,6 +39,45 @@ def test_scheduler_bit_exact(seed):
         assert np.array_equal(ns.cpu().numpy(), ns_ref), parts
 
 
+def test_scheduler_bit_exact_large_batch():
+    """More than 8192 requests: the scheduler keeps its prefix array in global memory instead of
+    shared memory and overwrites num_splits between its passes."""
+    import attention_mla_get_b200 as mla
+    rng = np.random.default_rng(7)
+    B = 9000
+    sl = rng.integers(0, 3000, size=B).astype(np.int32)
+    sl[rng.random(B) < 0.05] = 0
+    for parts in (1, 148, 1000):
+        md, ns = mla.mla_get_metadata(torch.from_numpy(sl).cuda(), 16, 1, num_sm_parts=parts)
+        md_ref, ns_ref = oracle.schedule(sl, parts)
+        assert np.array_equal(md.cpu().numpy(), md_ref), parts
+        assert np.array_equal(ns.cpu().numpy(), ns_ref), parts
+
+
+def test_scheduler_cost_overflow_is_flagged():
+    """A batch whose total cost (sum of ceil(L/128) + 2) reaches 2^31 does not fit the scheduler's
+    32-bit prefix sums: the metadata comes back empty and flagged, and a decode call given it
+    raises MLA_STATUS_BAD_METADATA and writes O = 0, LSE = -inf instead of reading the cache."""
+    import attention_mla_get_b200 as mla
+    B = 160
+    sl = np.full(B, 2**31 - 1, dtype=np.int32)      # 2^24 blocks each: total cost about 2.7e9
+    sl_d = torch.from_numpy(sl).cuda()
+    md, ns = mla.mla_get_metadata(sl_d, 16, 1, num_sm_parts=148)
+    md, ns = md.cpu().numpy(), ns.cpu().numpy()
+    assert (md[:, 5] == 1).all() and (md[:, 0] == B).all() and (md[:, 2] == B).all()
+    assert (ns == 0).all()
+    # a decode call with that metadata: a one-page cache that no part ever reads
+    q = torch.randn(B, 1, 16, 576, device="cuda").to(torch.bfloat16)
+    kv = torch.zeros(1, 64, 1, 576, dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros(B, 1, dtype=torch.int32, device="cuda")
+    md_d, ns_d = torch.from_numpy(md).cuda(), torch.from_numpy(ns).cuda()
+    ws = torch.zeros(mla.mla_workspace_size(B, 148, 16, 1), dtype=torch.uint8, device="cuda")
+    out, lse = mla.mla_decode_kvcache(q, kv, bt, sl_d, 512, md_d, ns_d, workspace=ws)
+    torch.cuda.synchronize()
+    assert mla.mla_read_status(ws) == 2
+    assert (out.float() == 0).all() and torch.isneginf(lse).all()
+
+
 def test_num_sm_parts_matches_rule():
     import attention_mla_get_b200 as mla
     sms = torch.cuda.get_device_properties(0).multi_processor_count
@@ -229,6 +268,33 @@ def test_fp8_small_scales(h_q):
     out, lse, status, _ = run_gpu(case)
     assert status == 0
     compare(case, out.astype(np.float64) * 2.0 ** 10, lse, O_ref * 2.0 ** 10, L_ref)
+
+
+def _bf16_bits(x):
+    return np.float32(x).view(np.uint32) >> 16
+
+
+@pytest.mark.parametrize("what", ["scale", "q", "rope", "none"])
+def test_fp8_pair_reports_f16_range(what):
+    """The CTA-pair FP8 path multiplies f16 operands; a value that leaves the f16 range raises
+    MLA_STATUS_F16_RANGE (4) instead of passing silently.  A group scale above 65504 / 448, a
+    q value of 70000, or a RoPE dim of 70000 in a token that exists each trigger it; NaN page
+    tails (never read into a result) and in-range data do not."""
+    case = mi.make_case(2, 1, 128, [300, 1000], kv_format="fp8", seed=58, poison=True, spare_blocks=2)
+    kv = case.kv.reshape(-1, 64, mi.FP8_TOKEN_BYTES)
+    blk = int(case.block_table[1, 3])          # request 1, tokens 192..255: all exist
+    if what == "scale":
+        sc = kv[blk, 5, 512:528].copy().view(np.float32)
+        sc[2] = np.float32(200.0)
+        kv[blk, 5, 512:528] = sc.view(np.uint8)
+    elif what == "rope":
+        r = kv[blk, 7, 528:656].copy().view(np.uint16)
+        r[11] = _bf16_bits(70000.0)
+        kv[blk, 7, 528:656] = r.view(np.uint8)
+    elif what == "q":
+        case.q_bits[0, 0, 77, 300] = _bf16_bits(70000.0)
+    out, lse, status, _ = run_gpu(case)
+    assert status == (0 if what == "none" else 4)
 
 
 def test_fp8_nan_in_unreadable_slots_does_not_leak():

@@ -1,8 +1,10 @@
 """mla_decode_kvcache_noalloc through the C-ABI: the decode call for callers that cannot
 allocate device memory (its workspace is a 16 MiB array inside libmla).  Its output must
 match the regular entry point's, within the tolerances of the other GPU tests, on two calls
-in a row (the second call reuses the array the first one left behind), and a problem whose
-workspace exceeds the array is rejected before anything runs.
+in a row (the second call reuses the array the first one left behind), and the fp64 oracle
+within the same tolerances; its device status word, read back with mla_noalloc_read_status,
+must be clear after each call; a problem whose workspace exceeds the array is rejected
+before anything runs.
 
 This file is collected last on purpose: it runs after every other test, and it also runs
 alone in a fresh process."""
@@ -14,6 +16,7 @@ import pytest
 import torch
 
 import mla_inputs as mi
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +31,15 @@ def _lib():
     L.mla_decode_kvcache_noalloc.argtypes = [vp, vp, i64, vp, i32, vp, i32, i32, i32, i32, i32, vp, i32, vp,
                                              ctypes.c_float, i32, i32, vp, vp, vp]
     L.mla_decode_kvcache_noalloc.restype = i32
+    L.mla_noalloc_read_status.argtypes = [i32, ctypes.POINTER(i32), vp]
+    L.mla_noalloc_read_status.restype = i32
     return L
+
+
+def _status(L):
+    v = ctypes.c_int(-1)
+    assert L.mla_noalloc_read_status(0, ctypes.byref(v), torch.cuda.current_stream().cuda_stream) == 0
+    return v.value
 
 
 def _noalloc(L, case, q, kv, bt, sl, md, ns, out, lse):
@@ -57,15 +68,20 @@ def test_noalloc_matches_regular_entry_point_twice(cuda_ok):
         ref_out, ref_lse = mla.mla_decode_kvcache(q, kv, bt, sl, 512, md, ns, softmax_scale=case.softmax_scale)
         ref_o = ref_out.float().cpu().numpy()
         ref_l = ref_lse.cpu().numpy()
+        o64, l64 = oracle.mla_decode_reference(case)
         for _ in range(2):
             out = torch.full_like(ref_out, float("nan"))
             lse = torch.full_like(ref_lse, float("nan"))
             assert _noalloc(L, case, q, kv, bt, sl, md, ns, out, lse) == 0
             torch.cuda.synchronize()
+            assert _status(L) == 0
             o, l = out.float().cpu().numpy(), lse.cpu().numpy()
             assert np.isfinite(o).all() and np.isfinite(l).all()
             assert np.all(np.abs(o - ref_o) <= 5e-3 + 1e-2 * np.abs(ref_o))
             assert np.abs(l - ref_l).max() <= 1e-3
+            # and directly against the fp64 oracle
+            assert np.all(np.abs(o - o64) <= 5e-3 + 1e-2 * np.abs(o64))
+            assert np.abs(l - l64).max() <= 1e-3
 
 
 def test_noalloc_rejects_problems_larger_than_its_scratch(cuda_ok):
