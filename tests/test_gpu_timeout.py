@@ -1,6 +1,6 @@
-"""The bounded-wait failure path of the single-CTA decode kernel, exercised without faulting or
-hanging the GPU: mla_fault_injection_arm makes the next call's copy producer skip one slot fill
-and shortens every pipeline wait to a few milliseconds.  The slot's consumer then waits in vain,
+"""The bounded-wait failure path of the single-CTA decode kernel (33 to 64 query rows per
+request), exercised without faulting or hanging the GPU: mla_fault_injection_arm makes the next
+call's copy producer skip one slot fill and shortens every pipeline wait to a few milliseconds.  The slot's consumer then waits in vain,
 the bound runs out, the kernel sets MLA_STATUS_WAIT_TIMEOUT in the workspace status word, every
 role of the CTA unwinds (copies in flight drained, tensor memory freed) and the call returns.
 A normal call that follows on the same stream must be correct and report no error."""
@@ -21,7 +21,7 @@ WAIT_LIMIT = 1 << 22   # SM clock cycles: about 2 ms at B200 clocks
 def test_withheld_fill_times_out_and_next_call_is_correct(cuda_ok, withhold):
     import attention_mla_get_b200 as mla
     # one part: the whole batch runs on one CTA, so fill indices up to 9 per 128-token step exist
-    case = mi.make_case(2, 1, 16, [1000, 300], seed=61)
+    case = mi.make_case(2, 1, 64, [1000, 300], seed=61)
     q, kv, bt, sl = to_device(case)
     md, ns = mla.mla_get_metadata(sl, case.rows, 1, num_sm_parts=1)
     ws = torch.zeros(mla.mla_workspace_size(case.batch, 1, case.rows, 1), dtype=torch.uint8, device="cuda")
@@ -46,7 +46,7 @@ def test_withheld_fill_times_out_and_next_call_is_correct(cuda_ok, withhold):
 def test_arm_is_taken_by_one_call_only(cuda_ok):
     """An armed setting applies to exactly one call: the call after it runs with the normal bound."""
     import attention_mla_get_b200 as mla
-    case = mi.make_case(1, 1, 16, [700], seed=62)
+    case = mi.make_case(1, 1, 64, [700], seed=62)
     q, kv, bt, sl = to_device(case)
     md, ns = mla.mla_get_metadata(sl, case.rows, 1, num_sm_parts=1)
     ws = torch.zeros(mla.mla_workspace_size(case.batch, 1, case.rows, 1), dtype=torch.uint8, device="cuda")
