@@ -177,9 +177,15 @@ def oracle_baseline(case, budget_s: float = 15.0):
 
 
 # DRAM bytes (read + write) per launch of the main kernel from an ncu capture of the current
-# kernel, scaled to the full workload by the KV bytes it processes (see profiles/); None when
-# the kernel has changed since the counters were taken.
-TRAFFIC = {"mem_b128_h16_L8192": 1253.8e6}
+# kernel, scaled to the full workload by the bytes it processes when the capture ran a smaller
+# batch (see profiles/); None when the kernel has changed since the counters were taken.
+TRAFFIC = {
+    "mem_b128_h16_L8192": 1237.9e6,            # batch 32 capture x 4.0
+    "varlen_b128_h128": 1263.8e6,              # batch 32 capture x 4.37
+    "causal_b64_sq2_h128": 361.4e6,            # full capture
+    "fp8_b128_h128_L16384": 1509.2e6,          # batch 16 capture x 8
+    "sparse_b128_h128_L8192_topk2048": 345.1e6,  # batch 32 capture x 4
+}
 
 
 def rank_case(workload: str, rank: int, batch=None):
@@ -509,7 +515,7 @@ def main():
                 "ms_per_step": ms_step, "decode_ms": wm["decode_ms"],
                 "gbs": wunits["bytes"] / (ms_step * 1e-3) / 1e9, "tflops": wunits["flops"] / (ms_step * 1e-3) / 1e12,
                 "steps": args.per_steps, "warmup": 3,
-                "roofline": roofline_of(wunits, wm["decode_ms"], ms_step, peaks),
+                "roofline": dict(roofline_of(wunits, wm["decode_ms"], ms_step, peaks), traffic=TRAFFIC.get(name)),
                 "clocks": wm["clocks"], "device_status": wm["status"],
                 "gpu_launches": 3 * args.per_steps,
                 "config": {"batch": wcase.batch, "s_q": wcase.s_q, "h_q": wcase.h_q, "causal": wcase.causal,
@@ -530,7 +536,7 @@ def main():
     tflops = units["flops"] * world * args.steps / (ms_total * 1e-3) / 1e12
     roof = roofline_of(units, decode_ms, ms_total / args.steps, peaks)
     roof["kernel"] = "mla_decode_kvcache (split-KV main + combine), decode calls alone"
-    roof["traffic"] = TRAFFIC.get(args.workload) if roof["bound"] == "hbm" else None
+    roof["traffic"] = TRAFFIC.get(args.workload)
     line = {
         "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
