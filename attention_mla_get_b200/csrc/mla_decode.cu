@@ -973,11 +973,10 @@ int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtenso
 
 }  // namespace
 
+// bf16 cache, 33 to 64 query rows (up to 32 run on the dim-split cluster, mla_decode_dsplit.cu)
 int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const OutMaps& om, const DecodeParams& p,
                        int rows_per_cta, cudaStream_t stream) {
   switch (rows_per_cta) {
-    case 16: return launch_impl<16, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
-    case 32: return launch_impl<32, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
     case 64: return launch_impl<64, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }
