@@ -410,6 +410,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // slot k: this CTA's dims d0 + 128k .. d0 + 128k + 127 (two 64-dim atoms, two pages)
             const int s = static_cast<int>(g % C::kNumSlots);
             const uint32_t use = g / C::kNumSlots;
+            if (rank == 0 && g + 1 == static_cast<uint32_t>(p.withhold_fill1)) {
+              // fault injection (tests only): CTA 0 never issues this fill, so its MMA thread's
+              // bounded wait runs out and both CTAs of the cluster unwind
+              ++g;
+              continue;
+            }
             if (!dwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) { ok = false; break; }
             mbar_arrive_expect_tx(bar(kBarSlotFull + s), 2u * npg * kBoxBytes);
             const uint32_t dst = sSlots + static_cast<uint32_t>(s) * kSlotBytes;

@@ -52,8 +52,8 @@ struct DecodeParams {
   int topk;
   int vq;
   int kv_len;             // sparse prefill: tokens of the one contiguous cache (cache_seqlens null)
-  // fault injection for tests of the bounded waits (mla_fault_injection_arm; single-CTA bf16
-  // kernel only): a shorter wait bound, and 1 + the index of a slot fill the producer skips
+  // fault injection for tests of the bounded waits (mla_fault_injection_arm; bf16 kernels up to
+  // 64 rows): a shorter wait bound, and 1 + the index of a slot fill the producer skips
   long long wait_limit;   // 0: the default bound
   int withhold_fill1;     // 0: none
 };

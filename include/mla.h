@@ -283,8 +283,10 @@ MLA_API int mla_session_destroy(mla_session* session);
  *                      waits in vain until the bound runs out, sets MLA_STATUS_WAIT_TIMEOUT,
  *                      and every role of the CTA unwinds (copies in flight are drained, tensor
  *                      memory is freed); the call's outputs are undefined.
- * Only the single-CTA bf16 kernel (33 to 64 query rows per request) honours the setting; the
- * next call takes and clears it whichever kernel it runs.  Errors: MLA_ERR_BAD_SHAPE for a
+ * Honoured by the bf16 kernels up to 64 query rows per request: the single CTA (33 to 64 rows)
+ * and the dim-split cluster (up to 32 rows; fill index counted in its first CTA, whose peer
+ * then unwinds through the cluster's abort flag).  The next call takes and clears the setting
+ * whichever kernel it runs.  Errors: MLA_ERR_BAD_SHAPE for a
  * negative limit or a fill index below -1.
  */
 MLA_API int mla_fault_injection_arm(long long wait_limit_cycles, int withhold_fill);
