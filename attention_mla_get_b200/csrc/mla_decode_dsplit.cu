@@ -451,6 +451,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       DualWalk walk(p, part0, has1);
       int b, c0, c1, split;
+      // shared-memory descriptors of the operands' first bytes; an operand at byte offset o from
+      // there is the descriptor plus o >> 4 (the 14-bit start-address field, 16-byte units)
+      const uint64_t kdesc0 = smem_desc(sSlots, 16, 1024, kSwizzle128);
+      const uint64_t vdesc0 = smem_desc(sSlots, kAtomBytes, 1024, kSwizzle128);
+      const uint64_t qdesc0 = smem_desc(sQ, 16, 1024, kSwizzle128);
+      const uint64_t rdesc0 = smem_desc(sRope, 16, 512, kSwizzle64);
+      const uint64_t qrdesc0 = smem_desc(sQ + 4 * C::kQAtomBytes, 16, 512, kSwizzle64);
+      const uint64_t pdesc0 = smem_desc(sP, 16 * 8 * C::kPRowBytes, 8 * C::kPRowBytes, C::kPLayout);
+      auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + static_cast<uint64_t>(bytes >> 4); };
       while (ok && walk.next(p, b, c0, c1, split)) {
         const int n = c1 - c0;
         if (!dwait(bar(kBarQFull), chunk & 1, wc)) break;
@@ -467,12 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = static_cast<int>(gr % kRopeSlots);
             if (!dwait(bar(kBarRopeFull + r), (gr / kRopeSlots) & 1u, wc)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t rbase = sRope + static_cast<uint32_t>(r) * kRopeSlotBytes;
+            const uint64_t rdesc = adv(rdesc0, static_cast<uint32_t>(r) * kRopeSlotBytes);
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk)
-              umma_bf16(d, smem_desc(rbase + 32 * kk, 16, 512, kSwizzle64),
-                        smem_desc(sQ + 4 * C::kQAtomBytes + 32 * kk, 16, 512, kSwizzle64), C::kIdescQK,
-                        kk != 0 ? 1u : 0u);
+              umma_bf16(d, adv(rdesc, 32 * kk), adv(qrdesc0, 32 * kk), C::kIdescQK, kk != 0 ? 1u : 0u);
             umma_commit(bar(kBarRopeEmpty + r));
             ++gr;
             for (int k = 0; ok && k < 2; ++k) {
@@ -480,14 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!dwait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) { ok = false; break; }
               tc_fence_after();
               ++g;
-              const uint32_t kbase = sSlots + s * kSlotBytes;
+              const uint64_t kdesc = adv(kdesc0, s * kSlotBytes);
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t a = kbase + (kk >> 2) * kAtomBytes + (kk & 3) * 32;
-                const uint32_t bq = sQ + (2 * k + (kk >> 2)) * C::kQAtomBytes + (kk & 3) * 32;
-                umma_bf16(d, smem_desc(a, 16, 1024, kSwizzle128), smem_desc(bq, 16, 1024, kSwizzle128), C::kIdescQK,
-                          1u);
-              }
+              for (int kk = 0; kk < 8; ++kk)
+                umma_bf16(d, adv(kdesc, (kk >> 2) * kAtomBytes + (kk & 3) * 32),
+                          adv(qdesc0, (2 * k + (kk >> 2)) * C::kQAtomBytes + (kk & 3) * 32), C::kIdescQK, 1u);
             }
             if (!ok) break;
             umma_commit(bar(kBarSFull + sb));
@@ -499,18 +503,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!dwait(bar(kBarPFull + pb), (up / kNumP) & 1u, wc)) { ok = false; break; }
             if (t == 0 && !dwait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t pbase = sP + static_cast<uint32_t>(pb) * C::kPBytes;
+            const uint64_t pdesc = adv(pdesc0, static_cast<uint32_t>(pb) * C::kPBytes);
             for (int k = 0; k < 2; ++k) {
               const uint32_t s = (gchunk + 2u * static_cast<uint32_t>(t) + static_cast<uint32_t>(k)) % C::kNumSlots;
-              const uint32_t vbase = sSlots + s * kSlotBytes;
+              const uint64_t vdesc = adv(vdesc0, s * kSlotBytes);
               const uint32_t d = tmem + C::kColO + k * RG;
 #pragma unroll
-              for (int kt = 0; kt < 8; ++kt) {
-                const uint64_t adesc = smem_desc(vbase + kt * 2048, kAtomBytes, 1024, kSwizzle128);
-                const uint64_t bdesc = smem_desc(pbase + kt * 16 * C::kPRowBytes, 16 * 8 * C::kPRowBytes,
-                                                 8 * C::kPRowBytes, C::kPLayout);
-                umma_bf16(d, adesc, bdesc, C::kIdescPV, (t == 0 && kt == 0) ? 0u : 1u);
-              }
+              for (int kt = 0; kt < 8; ++kt)
+                umma_bf16(d, adv(vdesc, kt * 2048), adv(pdesc, kt * 16 * C::kPRowBytes), C::kIdescPV,
+                          (t == 0 && kt == 0) ? 0u : 1u);
               umma_commit(bar(kBarSlotEmpty + s));
             }
             umma_commit(bar(kBarPEmpty + pb));
