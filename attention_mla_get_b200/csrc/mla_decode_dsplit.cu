@@ -441,7 +441,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 5) {
     // ================================ MMA issuer ==================================
-    if (lane == 0) {
+    // the whole warp runs the issue loop; every wait is observed by all lanes and its outcome made
+    // warp-uniform, each MMA and commit is issued by one elected lane
+    {
       uint32_t g = 0;   // slot fills consumed by QK
       uint32_t gr = 0;  // RoPE fills consumed
       uint32_t u = 0;   // steps whose QK was issued
@@ -462,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + static_cast<uint64_t>(bytes >> 4); };
       while (ok && walk.next(p, b, c0, c1, split)) {
         const int n = c1 - c0;
-        if (!dwait(bar(kBarQFull), chunk & 1, wc)) break;
+        if (!warp_all_dwait(bar(kBarQFull), chunk & 1, wc)) break;
         tc_fence_after();
         for (int e = 0; ok && e < 2 * n; ++e) {
           bool is_pv;
@@ -471,37 +473,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!is_pv) {
             // QK(t): partial S^T over this CTA's 288 dims into S buffer u % 2
             const int sb = static_cast<int>(u % kNumS);
-            if (!dwait(bar(kBarSEmpty + sb), ((u / kNumS) & 1u) ^ 1u, wc)) { ok = false; break; }
+            if (!warp_all_dwait(bar(kBarSEmpty + sb), ((u / kNumS) & 1u) ^ 1u, wc)) { ok = false; break; }
             const uint32_t d = tmem + C::kColS + sb * RG;
             const int r = static_cast<int>(gr % kRopeSlots);
-            if (!dwait(bar(kBarRopeFull + r), (gr / kRopeSlots) & 1u, wc)) { ok = false; break; }
+            if (!warp_all_dwait(bar(kBarRopeFull + r), (gr / kRopeSlots) & 1u, wc)) { ok = false; break; }
             tc_fence_after();
             const uint64_t rdesc = adv(rdesc0, static_cast<uint32_t>(r) * kRopeSlotBytes);
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk)
-              umma_bf16(d, adv(rdesc, 32 * kk), adv(qrdesc0, 32 * kk), C::kIdescQK, kk != 0 ? 1u : 0u);
-            umma_commit(bar(kBarRopeEmpty + r));
+              umma_bf16_warp(d, adv(rdesc, 32 * kk), adv(qrdesc0, 32 * kk), C::kIdescQK, kk != 0 ? 1u : 0u);
+            umma_commit_warp(bar(kBarRopeEmpty + r));
             ++gr;
             for (int k = 0; ok && k < 2; ++k) {
               const uint32_t s = g % C::kNumSlots;
-              if (!dwait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) { ok = false; break; }
+              if (!warp_all_dwait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) { ok = false; break; }
               tc_fence_after();
               ++g;
               const uint64_t kdesc = adv(kdesc0, s * kSlotBytes);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                umma_bf16(d, adv(kdesc, (kk >> 2) * kAtomBytes + (kk & 3) * 32),
+                umma_bf16_warp(d, adv(kdesc, (kk >> 2) * kAtomBytes + (kk & 3) * 32),
                           adv(qdesc0, (2 * k + (kk >> 2)) * C::kQAtomBytes + (kk & 3) * 32), C::kIdescQK, 1u);
             }
             if (!ok) break;
-            umma_commit(bar(kBarSFull + sb));
+            umma_commit_warp(bar(kBarSFull + sb));
             ++u;
-            if (t == n - 1) umma_commit(bar(kBarQEmpty));
+            if (t == n - 1) umma_commit_warp(bar(kBarQEmpty));
           } else {
             // PV(t): O_c^T += V_c^T . P^T from the two slots QK(t) read (kept since then)
             const int pb = static_cast<int>(up % kNumP);
-            if (!dwait(bar(kBarPFull + pb), (up / kNumP) & 1u, wc)) { ok = false; break; }
-            if (t == 0 && !dwait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) { ok = false; break; }
+            if (!warp_all_dwait(bar(kBarPFull + pb), (up / kNumP) & 1u, wc)) { ok = false; break; }
+            if (t == 0 && !warp_all_dwait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) { ok = false; break; }
             tc_fence_after();
             const uint64_t pdesc = adv(pdesc0, static_cast<uint32_t>(pb) * C::kPBytes);
             for (int k = 0; k < 2; ++k) {
@@ -510,21 +512,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t d = tmem + C::kColO + k * RG;
 #pragma unroll
               for (int kt = 0; kt < 8; ++kt)
-                umma_bf16(d, adv(vdesc, kt * 2048), adv(pdesc, kt * 16 * C::kPRowBytes), C::kIdescPV,
+                umma_bf16_warp(d, adv(vdesc, kt * 2048), adv(pdesc, kt * 16 * C::kPRowBytes), C::kIdescPV,
                           (t == 0 && kt == 0) ? 0u : 1u);
-              umma_commit(bar(kBarSlotEmpty + s));
+              umma_commit_warp(bar(kBarSlotEmpty + s));
             }
-            umma_commit(bar(kBarPEmpty + pb));
+            umma_commit_warp(bar(kBarPEmpty + pb));
             ++up;
           }
         }
         if (!ok) break;
-        umma_commit(bar(kBarOFull));
+        umma_commit_warp(bar(kBarOFull));
         gchunk += 2u * static_cast<uint32_t>(n);
         ++chunk;
       }
       // every MMA this thread issued is complete before TMEM is released
-      umma_commit(bar(kBarDrain));
+      umma_commit_warp(bar(kBarDrain));
       drain_wait(bar(kBarDrain), 0);
     }
   } else {
