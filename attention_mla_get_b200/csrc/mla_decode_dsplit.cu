@@ -22,7 +22,8 @@
 // one after the other, so num_sm_parts keeps its one-SM-per-part meaning.
 //
 // Roles per CTA: warps 0-3 softmax + epilogue (thread = token lane of S^T, then dim lane of
-// O^T), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner.  Issue order per chunk of n
+// O^T), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner (both run converged on the whole
+// warp, one elected lane issuing each copy, MMA and commit).  Issue order per chunk of n
 // steps: QK(0), QK(1), PV(0), QK(2), PV(1), ..., PV(n-1) (two S^T buffers in TMEM).  MMAs are
 // cta_group::1 (each CTA's tensor core works on its own dims); the only cross-CTA traffic is
 // the score exchange and, on a time-out, the abort flag.
@@ -370,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 4) {
     // ================================ TMA producer ================================
-    if (lane == 0) {
+    // the whole warp runs the fill loop; one elected lane issues each copy and arrive
+    {
       const uint64_t pol = policy_evict_first();  // every byte of the cache is read once
       uint32_t g = 0;   // slot fills issued
       uint32_t gr = 0;  // RoPE half-slot fills issued
@@ -386,10 +388,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int L = p.cache_seqlens[b];
         const int npages = (L + kPage - 1) / kPage;
         const int32_t* bt = p.block_table + static_cast<long long>(b) * p.max_blocks;
-        if (!dwait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(bar(kBarQFull), 4u * C::kQAtomBytes + C::kQRopeBytes);
-        for (int a = 0; a < 4; ++a) tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, d0 + 64 * a, 0, b, bar(kBarQFull));
-        tma_load_3d(sQ + 4 * C::kQAtomBytes, &tm_q_rope, dr, 0, b, bar(kBarQFull));
+        if (!warp_all_dwait(bar(kBarQEmpty), (q_fills & 1) ^ 1, wc)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(kBarQFull), 4u * C::kQAtomBytes + C::kQRopeBytes);
+          for (int a = 0; a < 4; ++a) tma_load_3d(sQ + a * C::kQAtomBytes, &tm_q, d0 + 64 * a, 0, b, bar(kBarQFull));
+          tma_load_3d(sQ + 4 * C::kQAtomBytes, &tm_q_rope, dr, 0, b, bar(kBarQFull));
+        }
         ++q_fills;
         for (int t = 0; ok && t < c1 - c0; ++t) {
           const StepPages sp = step_pages(bt, c0 + t, npages);
@@ -398,11 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this CTA's 32 RoPE dims of the step's tokens (QK^T only)
             const int r = static_cast<int>(gr % kRopeSlots);
             const uint32_t use = gr / kRopeSlots;
-            if (!dwait(bar(kBarRopeEmpty + r), (use & 1u) ^ 1u, wc)) { ok = false; break; }
-            mbar_arrive_expect_tx(bar(kBarRopeFull + r), npg * kRopeBoxBytes);
+            if (!warp_all_dwait(bar(kBarRopeEmpty + r), (use & 1u) ^ 1u, wc)) { ok = false; break; }
             const uint32_t dst = sRope + static_cast<uint32_t>(r) * kRopeSlotBytes;
-            tma_load_2d(dst, &tm_kv_rope, dr, sp.a * kPage, bar(kBarRopeFull + r), pol);
-            if (sp.has_b) tma_load_2d(dst + kRopeBoxBytes, &tm_kv_rope, dr, sp.b * kPage, bar(kBarRopeFull + r), pol);
+            if (elect_one()) {
+              mbar_arrive_expect_tx(bar(kBarRopeFull + r), npg * kRopeBoxBytes);
+              tma_load_2d(dst, &tm_kv_rope, dr, sp.a * kPage, bar(kBarRopeFull + r), pol);
+              if (sp.has_b) tma_load_2d(dst + kRopeBoxBytes, &tm_kv_rope, dr, sp.b * kPage, bar(kBarRopeFull + r), pol);
+            }
             last_rope[r] = static_cast<int>(use);
             ++gr;
           }
@@ -416,14 +422,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               ++g;
               continue;
             }
-            if (!dwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) { ok = false; break; }
-            mbar_arrive_expect_tx(bar(kBarSlotFull + s), 2u * npg * kBoxBytes);
+            if (!warp_all_dwait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) { ok = false; break; }
             const uint32_t dst = sSlots + static_cast<uint32_t>(s) * kSlotBytes;
-            for (int a = 0; a < 2; ++a) {
-              const int x = d0 + 128 * k + 64 * a;
-              tma_load_2d(dst + a * kAtomBytes, &tm_kv, x, sp.a * kPage, bar(kBarSlotFull + s), pol);
-              if (sp.has_b)
-                tma_load_2d(dst + a * kAtomBytes + kBoxBytes, &tm_kv, x, sp.b * kPage, bar(kBarSlotFull + s), pol);
+            if (elect_one()) {
+              mbar_arrive_expect_tx(bar(kBarSlotFull + s), 2u * npg * kBoxBytes);
+              for (int a = 0; a < 2; ++a) {
+                const int x = d0 + 128 * k + 64 * a;
+                tma_load_2d(dst + a * kAtomBytes, &tm_kv, x, sp.a * kPage, bar(kBarSlotFull + s), pol);
+                if (sp.has_b) tma_load_2d(dst + a * kAtomBytes + kBoxBytes, &tm_kv, x, sp.b * kPage, bar(kBarSlotFull + s), pol);
+              }
             }
             last_use[s] = static_cast<int>(use);
             ++g;
@@ -431,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (*abort_flag) {
-        // let every copy this thread started land before the CTA may exit
+        // let every copy this warp started land before the CTA may exit
         for (int s = 0; s < C::kNumSlots; ++s)
           if (last_use[s] >= 0) drain_wait(bar(kBarSlotFull + s), static_cast<uint32_t>(last_use[s]) & 1u);
         for (int r = 0; r < kRopeSlots; ++r)

@@ -687,7 +687,9 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ================================ MMA issuer (leader) =========================
-    if (leader && lane == 0) {
+    // the leader's whole warp runs the issue loop (waits seen by every lane, outcome warp-uniform);
+    // each MMA and commit is issued by one elected lane
+    if (leader) {
       uint32_t u = 0;   // QK steps issued
       uint32_t up = 0;  // PV steps issued
       uint32_t rope_used = 0;
@@ -699,7 +701,7 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
       uint32_t gs = 0, gph = 0;  // slot of the next fill to consume, and its phase parity
       auto next_slot = [&](uint32_t& s) -> bool {
         s = gs;
-        if (!pwait(bar(kBarSlotFull + s), gph, wc)) return false;
+        if (!warp_all_wait(bar(kBarSlotFull + s), gph, wc)) return false;
         if (++gs == static_cast<uint32_t>(kNumSlots)) {
           gs = 0;
           gph ^= 1u;
@@ -713,7 +715,7 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
         const int L = SPARSE ? 0 : p.cache_seqlens[b];
         const int n = (c1 - c0 + 1) / 2;
         // FP8: both CTAs' dequant warps have converted their Q halves to f16
-        if (!pwait(bar(FP8 ? kBarQReady : kBarQFull), chunk & 1, wc)) break;
+        if (!warp_all_wait(bar(FP8 ? kBarQReady : kBarQFull), chunk & 1, wc)) break;
         for (int e = 0; ok && e < 2 * n; ++e) {
           bool is_v;
           int t;
@@ -721,17 +723,17 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
           if (!is_v) {
             const int sb = static_cast<int>(u & 1u);
             // the softmax warps finished their tcgen05.ld of this buffer (wait::ld) before arriving
-            if (!pwait(bar(kBarSEmpty + sb), ((u >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
+            if (!warp_all_wait(bar(kBarSEmpty + sb), ((u >> 1) & 1u) ^ 1u, wc)) { ok = false; break; }
             const uint32_t d = tmem + kColS + 128u * sb;
             // RoPE dims first (they have their own slot), then the four 128-dim K stages
-            if (!pwait(bar(FP8 ? kBarRopeReady : kBarRopeFull), rope_used & 1u, wc)) { ok = false; break; }
+            if (!warp_all_wait(bar(FP8 ? kBarRopeReady : kBarRopeFull), rope_used & 1u, wc)) { ok = false; break; }
             ++rope_used;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              umma_bf16_pair(d, smem_desc(sRope + 32 * kk, 16, 1024, kSwizzle128),
+              umma_bf16_pair_warp(d, smem_desc(sRope + 32 * kk, 16, 1024, kSwizzle128),
                              smem_desc(sQ + 8 * kBoxBytes + 32 * kk, 16, 1024, kSwizzle128), kIdescQK,
                              kk != 0 ? 1u : 0u);
-            umma_commit_pair_mc(bar(kBarRopeEmpty), 0x3);
+            umma_commit_pair_mc_warp(bar(kBarRopeEmpty), 0x3);
             for (int j = 0; ok && j < kKFills; ++j) {
               uint32_t s;
               if (!next_slot(s)) { ok = false; break; }
@@ -740,17 +742,17 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
               const uint64_t b0 = smem_desc(sQ + 2 * j * kBoxBytes, 16, 1024, kSwizzle128);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                umma_bf16_pair(d, a0 + static_cast<uint64_t>(((kk >> 2) * kHalfBytes + 32 * (kk & 3)) >> 4),
+                umma_bf16_pair_warp(d, a0 + static_cast<uint64_t>(((kk >> 2) * kHalfBytes + 32 * (kk & 3)) >> 4),
                                b0 + static_cast<uint64_t>(((kk >> 2) * kBoxBytes + 32 * (kk & 3)) >> 4), kIdescQK, 1u);
-              umma_commit_pair_mc(bar(kBarSlotEmpty + s), 0x3);
+              umma_commit_pair_mc_warp(bar(kBarSlotEmpty + s), 0x3);
             }
             if (!ok) break;
-            umma_commit_pair_mc(bar(kBarSFull + sb), 0x3);
+            umma_commit_pair_mc_warp(bar(kBarSFull + sb), 0x3);
             ++u;
-            if (t == n - 1) umma_commit_pair_mc(bar(kBarQEmpty), 0x3);
+            if (t == n - 1) umma_commit_pair_mc_warp(bar(kBarQEmpty), 0x3);
           } else {
-            if (!pwait(bar(kBarPFull), up & 1u, wc)) { ok = false; break; }
-            if (t == 0 && !pwait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) { ok = false; break; }
+            if (!warp_all_wait(bar(kBarPFull), up & 1u, wc)) { ok = false; break; }
+            if (t == 0 && !warp_all_wait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) { ok = false; break; }
             // orders PV after the softmax warps' rescale of O^T (tcgen05.st) -- once per step: a
             // tcgen05 fence in the issue stream drains the MMA pipe, so none sits before
             // operands that only TMA or shared-memory stores produced
@@ -762,7 +764,7 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
                 uint32_t s;
                 if (!next_slot(s)) { ok = false; break; }
                 if (tail) {
-                  if (!pwait(bar(kBarZFull + s), (zpar >> s) & 1u, wc)) { ok = false; break; }
+                  if (!warp_all_wait(bar(kBarZFull + s), (zpar >> s) & 1u, wc)) { ok = false; break; }
                   zpar ^= 1u << s;
                 }
                 // half h = page 2 blk + h of the step (64 tokens x 128 dims, 64-dim boxes 8 KB apart)
@@ -770,24 +772,24 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
                 const uint64_t b0 = smem_desc(sP + 128 * blk * 128, kBoxBytes, 1024, kSwizzle128);
 #pragma unroll
                 for (int kt = 0; kt < 8; ++kt)
-                  umma_bf16_pair(tmem + kColO + 128u * m,
+                  umma_bf16_pair_warp(tmem + kColO + 128u * m,
                                  a0 + static_cast<uint64_t>(((kt >> 2) * kHalfBytes + 2048 * (kt & 3)) >> 4),
                                  b0 + static_cast<uint64_t>((16 * kt * 128) >> 4), kIdescPV,
                                  (t == 0 && blk == 0 && kt == 0) ? 0u : 1u);
-                umma_commit_pair_mc(bar(kBarSlotEmpty + s), 0x3);
+                umma_commit_pair_mc_warp(bar(kBarSlotEmpty + s), 0x3);
               }
             }
             if (!ok) break;
-            umma_commit_pair_mc(bar(kBarPEmpty), 0x3);
+            umma_commit_pair_mc_warp(bar(kBarPEmpty), 0x3);
             ++up;
           }
         }
         if (!ok) break;
-        umma_commit_pair_mc(bar(kBarOFull), 0x3);
+        umma_commit_pair_mc_warp(bar(kBarOFull), 0x3);
         ++chunk;
       }
       // every pair MMA is complete before tensor memory is released
-      umma_commit_pair(bar(kBarDrain));
+      umma_commit_pair_warp(bar(kBarDrain));
       drain_wait(bar(kBarDrain), 0);
     }
   } else if (SPARSE && warp == kWarpIndex) {
