@@ -189,6 +189,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// Every lane observes the phase; false on every lane if any gave up.
+__device__ __forceinline__ bool warp_all_wait(uint32_t bar, uint32_t parity, const WaitCtl& wc) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc) ? 1 : 0) != 0;
+}
+
 // Warp reduce-scatter over the 32 token lanes of N column values.  Afterwards lane l holds
 // the warp-wide reduction of column col_of(l, i) in v[i], i < max(1, N / 32).
 template <int N, bool MAX>
@@ -522,7 +527,9 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
     }
   } else if (warp == 5) {
     // ================================ MMA issuer ==================================
-    if (lane == 0) {
+    // the whole warp runs the issue loop (waits seen by every lane, outcome warp-uniform); each
+    // MMA and commit is issued by one elected lane
+    {
       uint32_t g = 0;   // slot fills consumed
       uint32_t u = 0;   // steps whose QK was issued (S^T buffers)
       uint32_t up = 0;  // steps whose PV was issued (P buffers)
@@ -532,7 +539,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       int b, c0, c1, split;
       auto next_slot = [&](uint32_t& s) -> bool {
         s = g % C::kNumSlots;
-        if (!mbar_wait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) return false;
+        if (!warp_all_wait(bar(kBarSlotFull + s), (g / C::kNumSlots) & 1u, wc)) return false;
         ++g;
         if (SPARSE) fence_proxy_async_smem();  // slots written by cp.async (generic proxy)
         tc_fence_after();
@@ -540,7 +547,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       };
       auto do_qk = [&]() -> bool {
         const int sb = static_cast<int>(u % kNumS);
-        if (!mbar_wait(bar(kBarSEmpty + sb), ((u / kNumS) & 1u) ^ 1u, wc)) return false;
+        if (!warp_all_wait(bar(kBarSEmpty + sb), ((u / kNumS) & 1u) ^ 1u, wc)) return false;
         tc_fence_after();
         const uint32_t d = tmem + C::kColS + sb * RG;
         for (int ks = 0; ks < 5; ++ks) {
@@ -551,19 +558,19 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
           for (int kk = 0; kk < nk; ++kk) {
             const uint32_t a = kbase + (kk >> 2) * C::kAtomColBytes + (kk & 3) * 32;
             const uint32_t bq = sQ + (2 * ks + (kk >> 2)) * C::kQAtomBytes + (kk & 3) * 32;
-            umma_bf16(d, smem_desc(a, 16, 1024, kSwizzle128), smem_desc(bq, 16, 1024, kSwizzle128), C::kIdescQK,
+            umma_bf16_warp(d, smem_desc(a, 16, 1024, kSwizzle128), smem_desc(bq, 16, 1024, kSwizzle128), C::kIdescQK,
                       (ks | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(bar(kBarSlotEmpty + s));
+          umma_commit_warp(bar(kBarSlotEmpty + s));
         }
-        umma_commit(bar(kBarSFull + sb));
+        umma_commit_warp(bar(kBarSFull + sb));
         ++u;
         return true;
       };
       auto do_pv = [&](bool first_of_chunk) -> bool {
         const int pb = static_cast<int>(up % C::kNumP);
-        if (!mbar_wait(bar(kBarPFull + pb), (up / C::kNumP) & 1u, wc)) return false;
-        if (first_of_chunk && !mbar_wait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) return false;
+        if (!warp_all_wait(bar(kBarPFull + pb), (up / C::kNumP) & 1u, wc)) return false;
+        if (first_of_chunk && !warp_all_wait(bar(kBarOEmpty), (chunk & 1) ^ 1, wc)) return false;
         tc_fence_after();
         const uint32_t pbase = sP + static_cast<uint32_t>(pb) * C::kPBytes;
         for (int vs = 0; vs < 4; ++vs) {
@@ -576,17 +583,17 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
             const uint64_t adesc = smem_desc(vbase + kt * 2048, C::kAtomColBytes, 1024, kSwizzle128);
             const uint64_t bdesc = smem_desc(pbase + kt * 16 * C::kPRowBytes, 16 * 8 * C::kPRowBytes,
                                              8 * C::kPRowBytes, C::kPLayout);
-            umma_bf16(d, adesc, bdesc, C::kIdescPV, (first_of_chunk && kt == 0) ? 0u : 1u);
+            umma_bf16_warp(d, adesc, bdesc, C::kIdescPV, (first_of_chunk && kt == 0) ? 0u : 1u);
           }
-          umma_commit(bar(kBarSlotEmpty + s));
+          umma_commit_warp(bar(kBarSlotEmpty + s));
         }
-        umma_commit(bar(kBarPEmpty + pb));
+        umma_commit_warp(bar(kBarPEmpty + pb));
         ++up;
         return true;
       };
       while (ok && walk.next(p, b, c0, c1, split)) {
         const int n = c1 - c0;
-        if (!mbar_wait(bar(kBarQFull), chunk & 1, wc)) break;
+        if (!warp_all_wait(bar(kBarQFull), chunk & 1, wc)) break;
         for (int e = 0; ok && e < order_len(n); ++e) {
           bool is_v;
           int t;
@@ -595,15 +602,15 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
             ok = do_pv(t == 0);
           } else {
             ok = do_qk();
-            if (ok && t == n - 1) umma_commit(bar(kBarQEmpty));
+            if (ok && t == n - 1) umma_commit_warp(bar(kBarQEmpty));
           }
         }
         if (!ok) break;
-        umma_commit(bar(kBarOFull));
+        umma_commit_warp(bar(kBarOFull));
         ++chunk;
       }
-      // every MMA this thread issued is complete before TMEM is released
-      umma_commit(bar(kBarDrain));
+      // every MMA this warp issued is complete before TMEM is released
+      umma_commit_warp(bar(kBarDrain));
       mbar_wait_drain(bar(kBarDrain), 0);
     }
   } else if (warp < 4) {

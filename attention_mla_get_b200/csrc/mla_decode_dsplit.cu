@@ -532,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         gchunk += 2u * static_cast<uint32_t>(n);
         ++chunk;
       }
-      // every MMA this thread issued is complete before TMEM is released
+      // every MMA this warp issued is complete before TMEM is released
       umma_commit_warp(bar(kBarDrain));
       drain_wait(bar(kBarDrain), 0);
     }

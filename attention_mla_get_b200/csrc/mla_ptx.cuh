@@ -174,21 +174,13 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// MMA issue is warp-collective here: the whole warp executes each call (converged, the same
+// arguments on every lane) and one lane chosen by elect.sync issues the instruction.  An issue
+// loop run by a converged warp on warp-uniform counters keeps its descriptors on the uniform
+// datapath that tcgen05 issue reads; the same loop run by one lane of a diverged warp issued
+// MMAs 7-15 % slower (16- to 64-row decode).
+//
 // D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 inputs, fp32 accumulate), one CTA.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Warp-collective forms: the whole warp executes the call (converged, same arguments on every
-// lane) and one lane chosen by elect.sync issues it.  An issue loop run by a converged warp on
-// warp-uniform counters keeps its descriptors on the uniform datapath that tcgen05 issue reads;
-// the same loop run by one lane of a diverged warp issued MMAs ~7 % slower in the 16-row decode.
 __device__ __forceinline__ void umma_bf16_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                uint32_t accumulate) {
   asm volatile(
@@ -200,18 +192,13 @@ __device__ __forceinline__ void umma_bf16_warp(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// Arrive (once) on an mbarrier when every tcgen05.mma issued so far by this warp is done.
 __device__ __forceinline__ void umma_commit_warp(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 l;\n\t"
       "elect.sync l|e, 0xffffffff;\n\t"
       "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
       : "memory");
-}
-
-// Arrive (once) on an mbarrier when every tcgen05.mma issued so far by this thread is done.
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -367,27 +354,8 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 
 // D (+)= A * B over the pair: M rows split 128/128 over the two CTAs' A tiles and D (each SM's
 // tensor memory holds its M half x all N), N split in halves over the two CTAs' B tiles.
-// Issued by one thread of the leader CTA; descriptors address the same offsets in both CTAs.
-__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                               uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once, on the mbarrier at the same offset in every CTA of `cta_mask`, when every pair
-// MMA issued so far by this thread is complete.
-__device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-      "h"(cta_mask)
-      : "memory");
-}
-
-// Warp-collective forms of the three calls above (see umma_bf16_warp).
+// Issued by the leader CTA's MMA warp (warp-collective, see umma_bf16_warp); descriptors
+// address the same offsets in both CTAs.
 __device__ __forceinline__ void umma_bf16_pair_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                     uint32_t accumulate) {
   asm volatile(
@@ -399,6 +367,8 @@ __device__ __forceinline__ void umma_bf16_pair_warp(uint32_t d_tmem, uint64_t a_
       : "memory");
 }
 
+// Arrive once, on the mbarrier at the same offset in every CTA of `cta_mask`, when every pair
+// MMA issued so far by this warp is complete.
 __device__ __forceinline__ void umma_commit_pair_mc_warp(uint32_t bar, uint16_t cta_mask) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 l;\n\t"
@@ -408,6 +378,7 @@ __device__ __forceinline__ void umma_commit_pair_mc_warp(uint32_t bar, uint16_t 
       : "memory");
 }
 
+// Same, on one barrier of this CTA.
 __device__ __forceinline__ void umma_commit_pair_warp(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 l;\n\t"
@@ -416,7 +387,8 @@ __device__ __forceinline__ void umma_commit_pair_warp(uint32_t bar) {
       : "memory");
 }
 
-// Warp-collective: one elected lane runs `f` (an issue of a copy, an arrive); the warp stays converged.
+// Warp-collective: true on one lane chosen by elect.sync (the lane that issues a copy or an
+// arrive for the converged warp).
 __device__ __forceinline__ bool elect_one() {
   uint32_t e;
   asm volatile(
@@ -425,12 +397,6 @@ __device__ __forceinline__ bool elect_one() {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(e));
   return e != 0;
-}
-
-// Same, on one barrier of this CTA.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
 }
 
 // ------------------------------------------------------------------------------------
