@@ -182,14 +182,8 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-// Lane 0 waits, the warp learns the outcome.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtl& wc, int lane) {
-  int ok = 1;
-  if (lane == 0) ok = mbar_wait(bar, parity, wc) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
-// Every lane observes the phase; false on every lane if any gave up.
+// Every lane polls the barrier itself and the outcome is warp-uniform (false on every lane if
+// any gave up).  One polling lane plus a shuffle of the outcome measured slower.
 __device__ __forceinline__ bool warp_all_wait(uint32_t bar, uint32_t parity, const WaitCtl& wc) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc) ? 1 : 0) != 0;
 }
@@ -394,7 +388,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       auto fill = [&](int dims0, int natoms) -> bool {
         const int s = static_cast<int>(g % C::kNumSlots);
         const uint32_t use = g / C::kNumSlots;
-        if (!warp_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc, lane)) return false;
+        if (!warp_all_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc)) return false;
         const uint32_t dst = sSlots + static_cast<uint32_t>(s) * C::kSlotBytes;
         const int cpr = 8 * natoms;        // chunks per row slice
         const int rpi = 32 / cpr;          // rows per warp instruction
@@ -639,7 +633,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
         const int t0 = (c0 + t) * kBlockTokens;
         const int j = t0 + tid;
         const int sb = static_cast<int>(u % kNumS);
-        bool ok = warp_wait(bar(kBarSFull + sb), (u / kNumS) & 1u, wc, lane);
+        bool ok = warp_all_wait(bar(kBarSFull + sb), (u / kNumS) & 1u, wc);
         float x[RG];
         tc_fence_after();
 #pragma unroll
@@ -703,7 +697,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
         // P^T row of this token (bf16), once PV(u - kNumP) has released the buffer
         const int pb = static_cast<int>(u % C::kNumP);
         if (u >= static_cast<uint32_t>(C::kNumP))
-          ok &= warp_wait(bar(kBarPEmpty + pb), ((u - C::kNumP) / C::kNumP) & 1u, wc, lane);
+          ok &= warp_all_wait(bar(kBarPEmpty + pb), ((u - C::kNumP) / C::kNumP) & 1u, wc);
         {
           const uint32_t prow = static_cast<uint32_t>(tid) * C::kPRowBytes;
           const uint32_t pbase = sP + static_cast<uint32_t>(pb) * C::kPBytes;
@@ -718,7 +712,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
         if (rescale) {
           // O^T *= alpha per row, after PV(u - 1) has finished
           const uint32_t uq = u - 1;
-          ok &= warp_wait(bar(kBarPEmpty + uq % C::kNumP), (uq / C::kNumP) & 1u, wc, lane);
+          ok &= warp_all_wait(bar(kBarPEmpty + uq % C::kNumP), (uq / C::kNumP) & 1u, wc);
           tc_fence_after();
 #pragma unroll
           for (int vs = 0; vs < 4; ++vs) {
@@ -741,7 +735,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
           for (int vs = 0; vs < 4; ++vs) {
             const uint32_t gv = gchunk + slots_before_v(t, n) + vs;
             const uint32_t s = gv % C::kNumSlots;
-            ok &= warp_wait(bar(kBarSlotFull + s), (gv / C::kNumSlots) & 1u, wc, lane);
+            ok &= warp_all_wait(bar(kBarSlotFull + s), (gv / C::kNumSlots) & 1u, wc);
             if (j >= L) {
               const uint32_t rowaddr = sSlots + s * C::kSlotBytes + static_cast<uint32_t>(tid) * 128u;
 #pragma unroll
@@ -783,7 +777,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
 #pragma unroll
       for (int i = 0; i < C::kNOut; ++i) lsum[i] = 0.f;
       named_bar_sync(1, 128);
-      const bool ok = warp_wait(bar(kBarOFull), chunk & 1, wc, lane);
+      const bool ok = warp_all_wait(bar(kBarOFull), chunk & 1, wc);
       fail |= !ok;
       tc_fence_after();
       {
@@ -861,8 +855,8 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       auto dequant_slot = [&](int grp, uint32_t sbuf, int t0, int L) -> bool {
         const uint32_t s = gs % C::kNumSlots;
         const uint32_t r = gr % C::kNumRaw;
-        ok &= warp_wait(bar(kBarRawFull + r), (gr / C::kNumRaw) & 1u, wc, lane);
-        ok &= warp_wait(bar(kBarSlotEmpty + s), ((gs / C::kNumSlots) & 1u) ^ 1u, wc, lane);
+        ok &= warp_all_wait(bar(kBarRawFull + r), (gr / C::kNumRaw) & 1u, wc);
+        ok &= warp_all_wait(bar(kBarSlotEmpty + s), ((gs / C::kNumSlots) & 1u) ^ 1u, wc);
         const uint32_t dst = sSlots + s * C::kSlotBytes + static_cast<uint32_t>(dt) * 128u;
         const uint32_t swz = static_cast<uint32_t>(dt & 7);
         if (t0 + dt < L) {
@@ -930,7 +924,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
           const int t0 = (c0 + t) * kBlockTokens;
           const uint32_t su = us0 + static_cast<uint32_t>(t);  // scale fill of step t
           if (!is_v) {
-            ok &= warp_wait(bar(kBarScaleFull + su % kNumS), (su / kNumS) & 1u, wc, lane);
+            ok &= warp_all_wait(bar(kBarScaleFull + su % kNumS), (su / kNumS) & 1u, wc);
             ++us;
           }
           for (int grp = 0; grp < 4 && !aborted; ++grp) aborted = !dequant_slot(grp, su % kNumS, t0, L);

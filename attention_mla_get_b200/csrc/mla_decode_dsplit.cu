@@ -215,14 +215,8 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// Lane 0 waits, the warp learns the outcome.
-__device__ __forceinline__ bool warp_dwait(uint32_t bar, uint32_t parity, const DsCtl& c, int lane) {
-  int ok = 1;
-  if (lane == 0) ok = dwait(bar, parity, c) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
-// Every lane observes the phase itself (it then reads what the phase guards).
+// Every lane polls the barrier itself (it then reads what the phase guards); the outcome is
+// warp-uniform.  One polling lane plus a shuffle of the outcome measured slower.
 __device__ __forceinline__ bool warp_all_dwait(uint32_t bar, uint32_t parity, const DsCtl& c) {
   return __all_sync(0xffffffffu, dwait(bar, parity, c) ? 1 : 0) != 0;
 }
@@ -561,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = t0 + tid;
         const int sb = static_cast<int>(u % kNumS);
         const int xb = static_cast<int>(u % kNumX);
-        bool ok = warp_dwait(bar(kBarSFull + sb), (u / kNumS) & 1u, wc, lane);
+        bool ok = warp_all_dwait(bar(kBarSFull + sb), (u / kNumS) & 1u, wc);
         float x[RG];
         tc_fence_after();
 #pragma unroll
@@ -649,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P^T row of this token (bf16), once PV(u - kNumP) has released the buffer
         const int pb = static_cast<int>(u % kNumP);
         if (u >= static_cast<uint32_t>(kNumP))
-          ok &= warp_dwait(bar(kBarPEmpty + pb), ((u - kNumP) / kNumP) & 1u, wc, lane);
+          ok &= warp_all_dwait(bar(kBarPEmpty + pb), ((u - kNumP) / kNumP) & 1u, wc);
         {
           const uint32_t prow = static_cast<uint32_t>(tid) * C::kPRowBytes;
           const uint32_t pbase = sP + static_cast<uint32_t>(pb) * C::kPBytes;
@@ -664,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (rescale) {
           // O^T *= alpha per row, after PV(u - 1) has finished
           const uint32_t uq = u - 1;
-          ok &= warp_dwait(bar(kBarPEmpty + uq % kNumP), (uq / kNumP) & 1u, wc, lane);
+          ok &= warp_all_dwait(bar(kBarPEmpty + uq % kNumP), (uq / kNumP) & 1u, wc);
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
@@ -719,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       lsum = 0.f;
       named_bar_sync(1, 128);
-      const bool ok = warp_dwait(bar(kBarOFull), chunk & 1, wc, lane);
+      const bool ok = warp_all_dwait(bar(kBarOFull), chunk & 1, wc);
       fail |= !ok;
       tc_fence_after();
       {
