@@ -155,13 +155,10 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   EncodeTiledFn encode = encode_fn();
   if (!encode) return MLA_ERR_CUDA;
   const bool pair = mla::use_pair_kernel(rows, kv_dtype == MLA_KV_FP8);
-  // up to 32 rows over a bf16 cache: the dim-split cluster (each CTA half of the cached dims)
-  const bool dsplit = kv_dtype == MLA_KV_BF16 && rows <= mla::kDsplitRows;
   const int rg = pair ? mla::kRowsPerCta : rows_per_cta_for(rows);  // query rows of one Q box
 
   // q as a 3-D tensor {576 dims, rows, batch}; one box = 64 dims x rg rows of one request
-  // (and, for the dim-split cluster, 32 RoPE dims x rg rows with the 64-byte swizzle)
-  CUtensorMap tm_q, tm_q_rope, tm_kv, tm_kv_rope, tm_scale, tm_rope;
+  CUtensorMap tm_q, tm_kv, tm_scale, tm_rope;
   {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(rows),
                           static_cast<cuuint64_t>(batch)};
@@ -172,15 +169,9 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MLA_ERR_CUDA;
-    cuuint32_t box_rope[3] = {32, static_cast<cuuint32_t>(rg), 1};
-    if (dsplit && encode(&tm_q_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides,
-                         box_rope, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return MLA_ERR_CUDA;
   }
   if (kv_dtype == MLA_KV_BF16) {
-    // the cache as 2-D {576 dims, num_blocks * 64 tokens}; one box = 64 dims x one page (and,
-    // for the dim-split cluster, 32 RoPE dims x one page with the 64-byte swizzle)
+    // the cache as 2-D {576 dims, num_blocks * 64 tokens}; one box = 64 dims x one page
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDqk), static_cast<cuuint64_t>(num_blocks) * kPage};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDqk) * 2};
     cuuint32_t box[2] = {64, 64};
@@ -188,11 +179,6 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
     if (encode(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kvcache), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return MLA_ERR_CUDA;
-    cuuint32_t box_rope[2] = {32, 64};
-    if (dsplit && encode(&tm_kv_rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kvcache), dims, strides,
-                         box_rope, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return MLA_ERR_CUDA;
   } else {
     // FP8 tokens as a 2-D byte tensor {656 bytes, num_blocks * 64 tokens}, read three ways:
@@ -241,10 +227,8 @@ int mla_decode_kvcache(const void* q, const void* kvcache, int64_t num_blocks, c
   if (!encode_out_maps(encode, &om, p.o_part, out, rows, batch, num_sm_parts, rg == 16 ? 16 : 32))
     return MLA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int e = kv_dtype == MLA_KV_BF16 ? (pair     ? mla::launch_decode_pair_bf16(tm_q, tm_kv, om, p, st)
-                                     : dsplit ? mla::launch_decode_dsplit_bf16(tm_q, tm_q_rope, tm_kv, tm_kv_rope,
-                                                                               om, p, rg, st)
-                                              : mla::launch_decode_bf16(tm_q, tm_kv, om, p, rg, st))
+  int e = kv_dtype == MLA_KV_BF16 ? (pair ? mla::launch_decode_pair_bf16(tm_q, tm_kv, om, p, st)
+                                          : mla::launch_decode_bf16(tm_q, tm_kv, om, p, rg, st))
           : pair ? mla::launch_decode_pair_fp8(tm_q, tm_kv, tm_scale, tm_rope, om, p, st)
                  : mla::launch_decode_fp8(tm_q, tm_kv, tm_scale, tm_rope, om, p, rg, st);
   if (e != 0) return MLA_ERR_CUDA;

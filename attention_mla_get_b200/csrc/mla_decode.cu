@@ -10,15 +10,17 @@
 // of every tcgen05 MMA and the query rows are the N side:
 //   S^T [128 tokens x RG rows]  = K_tile[128 x 576]  . Q^T[576 x RG]      (fp32 in TMEM)
 //   O^T [512 dims  x RG rows] += V_tile^T[512 x 128] . P^T[128 x RG]      (fp32 in TMEM)
-// One CTA carries RG <= 64 query rows (R = 128 / 256 uses 2 / 4 CTAs on the same pages),
-// so O^T needs only 4*RG TMEM columns and the whole 512-dim output stays in TMEM.
+// One CTA carries RG = 16, 32 or 64 query rows (more rows per request run on the CTA pair of
+// mla_decode_pair.cu), so O^T needs only 4*RG TMEM columns and the whole 512-dim output stays
+// in TMEM.
 // A step covers 128 tokens (two 64-token pages).  Pages are TMA-loaded through the block
 // table in 64x64 boxes (the 9-boxes-per-page split on the wmrh.cn page, "内存访问优化策略")
 // into 32 KB ring slots (128 tokens x 128 dims, 128-byte swizzle).  The same slot layout is
 // read K-major by QK^T and MN-major (as V^T) by PV, so V is never transposed.
 //
 // Roles: warps 0-3 online softmax + epilogue (thread = token lane of S^T, then dim lane of
-// O^T), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner, warps 6-9 FP8 dequant.
+// O^T), warp 4 TMA producer (one lane), warp 5 MMA issuer and TMEM owner (the whole warp,
+// converged, one elected lane issuing each MMA and commit), warps 6-9 FP8 dequant.
 // Online softmax keeps a per-row running reference max (log2 units) and rescales O^T in
 // TMEM only when a block max exceeds it by more than kTau (the running-max-and-scale idea
 // of the wmrh.cn page, "跷跷板调度算法" paragraph); P^T is written to shared memory as
@@ -974,10 +976,12 @@ int launch_impl(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const CUtenso
 
 }  // namespace
 
-// bf16 cache, 33 to 64 query rows (up to 32 run on the dim-split cluster, mla_decode_dsplit.cu)
+// bf16 cache, up to 64 query rows (16-, 32- or 64-row tiles)
 int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const OutMaps& om, const DecodeParams& p,
                        int rows_per_cta, cudaStream_t stream) {
   switch (rows_per_cta) {
+    case 16: return launch_impl<16, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
+    case 32: return launch_impl<32, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
     case 64: return launch_impl<64, false>(tm_q, tm_kv, tm_kv, tm_kv, om, p, stream);
     default: return static_cast<int>(cudaErrorInvalidValue);
   }

@@ -92,12 +92,6 @@ int launch_scheduler(const int32_t* cache_seqlens, int batch, int num_sm_parts, 
                      int32_t* num_splits, cudaStream_t stream, int uniform_len = 0);
 int launch_decode_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const OutMaps& om, const DecodeParams& p,
                        int rows_per_cta, cudaStream_t stream);
-// up to 32 query rows, bf16 cache: a cluster of two CTAs splitting the cached dims
-// (tm_q_rope / tm_kv_rope: boxes of 32 RoPE dims with the 64-byte swizzle)
-int launch_decode_dsplit_bf16(const CUtensorMap& tm_q, const CUtensorMap& tm_q_rope, const CUtensorMap& tm_kv,
-                              const CUtensorMap& tm_kv_rope, const OutMaps& om, const DecodeParams& p,
-                              int rows_per_cluster, cudaStream_t stream);
-constexpr int kDsplitRows = 32;  // query rows up to which the dim-split cluster runs
 int launch_decode_fp8(const CUtensorMap& tm_q, const CUtensorMap& tm_codes, const CUtensorMap& tm_scale,
                       const CUtensorMap& tm_rope, const OutMaps& om, const DecodeParams& p, int rows_per_cta,
                       cudaStream_t stream);

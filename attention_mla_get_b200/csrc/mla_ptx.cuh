@@ -387,18 +387,6 @@ __device__ __forceinline__ void umma_commit_pair_warp(uint32_t bar) {
       : "memory");
 }
 
-// Warp-collective: true on one lane chosen by elect.sync (the lane that issues a copy or an
-// arrive for the converged warp).
-__device__ __forceinline__ bool elect_one() {
-  uint32_t e;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b32 l;\n\t"
-      "elect.sync l|p, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(e));
-  return e != 0;
-}
-
 // ------------------------------------------------------------------------------------
 // shared-memory matrix descriptors (tcgen05 format: start, LBO, SBO in 16-byte units,
 // version 1 at bits 46-47, layout type at bits 61-63)

@@ -283,9 +283,8 @@ MLA_API int mla_session_destroy(mla_session* session);
  *                      waits in vain until the bound runs out, sets MLA_STATUS_WAIT_TIMEOUT,
  *                      and every role of the CTA unwinds (copies in flight are drained, tensor
  *                      memory is freed); the call's outputs are undefined.
- * Honoured by the bf16 kernels up to 64 query rows per request: the single CTA (33 to 64 rows)
- * and the dim-split cluster (up to 32 rows; fill index counted in its first CTA, whose peer
- * then unwinds through the cluster's abort flag).  The next call takes and clears the setting
+ * Honoured by the single-CTA kernel, which runs bf16 caches with up to 64 query rows per
+ * request (fill index counted over the CTA).  The next call takes and clears the setting
  * whichever kernel it runs.  Errors: MLA_ERR_BAD_SHAPE for a
  * negative limit or a fill index below -1.
  */

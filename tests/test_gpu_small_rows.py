@@ -1,10 +1,9 @@
-"""GPU parity of the dim-split cluster (up to 32 query rows over a bf16 cache: two CTAs that
-each hold half of the 576 cached dims and exchange partial scores) against the fp64 oracle,
-on the cases that exercise what is specific to it: both CTAs' halves of the output, the
-exchange at every step, a cluster that walks two scheduler parts (or one, when the part count
-is odd), requests that end inside a step or have no second page, requests with no tokens,
-causal rows that see nothing, NaN in unreadable cache slots, and row counts that leave part of
-the 16- or 32-row tile empty.  Tolerances as in test_gpu_decode.py."""
+"""GPU parity of decode with up to 32 query rows over a bf16 cache (the single-CTA kernel's 16-
+and 32-row tiles; the memory-bound shape) against the fp64 oracle: row counts that leave part of
+the tile empty, requests that end inside a page or a step or have no second page, requests with
+no tokens, causal rows that see nothing, NaN in unreadable cache slots, scheduler part counts
+from one to more than there are steps (empty parts), split-count invariance and the block
+table's permutation invariance.  Tolerances as in test_gpu_decode.py."""
 import numpy as np
 import pytest
 
@@ -35,7 +34,7 @@ def test_row_counts(h_q, s_q, causal):
 
 @pytest.mark.parametrize("parts", [1, 2, 3, 7, 148, 149])
 def test_part_counts(parts):
-    # odd counts leave the last cluster a single part; more parts than steps leave parts empty
+    # more parts than steps leave parts empty
     case = mi.make_case(3, 1, 16, [4000, 300, 2100], seed=90)
     O_ref, L_ref = oracle.mla_decode_reference(case)
     out, lse, status, (md, ns) = run_gpu(case, num_sm_parts=parts)
