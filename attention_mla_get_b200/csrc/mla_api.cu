@@ -97,7 +97,8 @@ const char* mla_strerror(int code) {
                                    "s_q*h_q <= 4096 and num_blocks*64 < 2^31";
     case MLA_ERR_BAD_PARTS: return "num_sm_parts must be >= 1";
     case MLA_ERR_NO_DEVICE: return "CUDA device query failed";
-    case MLA_ERR_SCRATCH_LIMIT: return "the problem's workspace exceeds the 16 MiB built-in scratch of the no-alloc call";
+    case MLA_ERR_SCRATCH_LIMIT:
+      return "the problem's workspace exceeds the 16 MiB built-in scratch of the no-alloc call";
     case MLA_ERR_CUDA: return "a CUDA call failed";
     default: return "unknown libmla error code";
   }
@@ -253,8 +254,8 @@ int mla_get_metadata_sparse(int batch, int s_q, int topk, int h_q, int h_kv, int
   if (batch < 1 || s_q < 1 || topk < 1 || h_q < 1 || h_q > kMaxRows) return MLA_ERR_BAD_SHAPE;
   if (static_cast<long long>(batch) * s_q >= (1ll << 30)) return MLA_ERR_BAD_SHAPE;
   // the scheduler's 32-bit prefix sums: total cost = positions * (blocks of topk + 2) < 2^31
-  const long long cost = static_cast<long long>(batch) * s_q *
-                         ((static_cast<long long>(topk) + mla::kBlockTokens - 1) / mla::kBlockTokens + mla::kFixedSplitCost);
+  const long long blocks = (static_cast<long long>(topk) + mla::kBlockTokens - 1) / mla::kBlockTokens;
+  const long long cost = static_cast<long long>(batch) * s_q * (blocks + mla::kFixedSplitCost);
   if (cost >= (1ll << 31)) return MLA_ERR_BAD_SHAPE;
   if (h_kv != 1) return MLA_ERR_BAD_HEADS;
   if (num_sm_parts < 1) return MLA_ERR_BAD_PARTS;

@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
             const uint32_t a = kbase + (kk >> 2) * C::kAtomColBytes + (kk & 3) * 32;
             const uint32_t bq = sQ + (2 * ks + (kk >> 2)) * C::kQAtomBytes + (kk & 3) * 32;
             umma_bf16_warp(d, smem_desc(a, 16, 1024, kSwizzle128), smem_desc(bq, 16, 1024, kSwizzle128), C::kIdescQK,
-                      (ks | kk) != 0 ? 1u : 0u);
+                           (ks | kk) != 0 ? 1u : 0u);
           }
           umma_commit_warp(bar(kBarSlotEmpty + s));
         }

@@ -726,8 +726,8 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               umma_bf16_pair_warp(d, smem_desc(sRope + 32 * kk, 16, 1024, kSwizzle128),
-                             smem_desc(sQ + 8 * kBoxBytes + 32 * kk, 16, 1024, kSwizzle128), kIdescQK,
-                             kk != 0 ? 1u : 0u);
+                                  smem_desc(sQ + 8 * kBoxBytes + 32 * kk, 16, 1024, kSwizzle128), kIdescQK,
+                                  kk != 0 ? 1u : 0u);
             umma_commit_pair_mc_warp(bar(kBarRopeEmpty), 0x3);
             for (int j = 0; ok && j < kKFills; ++j) {
               uint32_t s;
@@ -738,7 +738,8 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
                 umma_bf16_pair_warp(d, a0 + static_cast<uint64_t>(((kk >> 2) * kHalfBytes + 32 * (kk & 3)) >> 4),
-                               b0 + static_cast<uint64_t>(((kk >> 2) * kBoxBytes + 32 * (kk & 3)) >> 4), kIdescQK, 1u);
+                                    b0 + static_cast<uint64_t>(((kk >> 2) * kBoxBytes + 32 * (kk & 3)) >> 4),
+                                    kIdescQK, 1u);
               umma_commit_pair_mc_warp(bar(kBarSlotEmpty + s), 0x3);
             }
             if (!ok) break;
@@ -768,9 +769,9 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
 #pragma unroll
                 for (int kt = 0; kt < 8; ++kt)
                   umma_bf16_pair_warp(tmem + kColO + 128u * m,
-                                 a0 + static_cast<uint64_t>(((kt >> 2) * kHalfBytes + 2048 * (kt & 3)) >> 4),
-                                 b0 + static_cast<uint64_t>((16 * kt * 128) >> 4), kIdescPV,
-                                 (t == 0 && blk == 0 && kt == 0) ? 0u : 1u);
+                                      a0 + static_cast<uint64_t>(((kt >> 2) * kHalfBytes + 2048 * (kt & 3)) >> 4),
+                                      b0 + static_cast<uint64_t>((16 * kt * 128) >> 4), kIdescPV,
+                                      (t == 0 && blk == 0 && kt == 0) ? 0u : 1u);
                 umma_commit_pair_mc_warp(bar(kBarSlotEmpty + s), 0x3);
               }
             }
