@@ -1080,8 +1080,12 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
           }
           if (kb >= c1 || j >= L) cmin = 1 << 30;
         }
+        // raw scores: the scale is applied in the exponent (ex2(S * scale - m)) and to the block
+        // maxima; the mask pass runs only when one of the warp's tokens is masked
+        if (__any_sync(0xffffffffu, cmin > -(1 << 30))) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = (c >= cmin) ? x[c] * p.scale_log2 : NEG_INF;
+          for (int c = 0; c < 64; ++c) x[c] = (c >= cmin) ? x[c] : NEG_INF;
+        }
         // column maxima over this warp's 32 tokens; lane l keeps columns l and 32 + l
         float k0 = NEG_INF, k1 = NEG_INF;
 #pragma unroll
@@ -1098,7 +1102,8 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
         if (tid < kRows) {
           // block max of row tid over this CTA's tokens, then over the pair's
           const float bm_own =
-              fmaxf(fmaxf(red[tid], red[kRows + tid]), fmaxf(red[2 * kRows + tid], red[3 * kRows + tid]));
+              fmaxf(fmaxf(red[tid], red[kRows + tid]), fmaxf(red[2 * kRows + tid], red[3 * kRows + tid])) *
+              p.scale_log2;
           const uint32_t xb = u & 1u;
           st_async_f32(other(sMisc + kMiscXMax + 4u * (xb * kRows + tid)), bm_own, other(bar(kBarMaxFull + xb)));
           if (tid == 0) mbar_arrive_expect_tx(bar(kBarMaxFull + xb), 4u * kRows);
@@ -1119,10 +1124,10 @@ __global__ void __launch_bounds__(PairCfg<FP8, SPARSE>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
           const float4 m4 = *reinterpret_cast<const float4*>(m_sm + 64 * h + c);
-          x[c + 0] = ex2(x[c + 0] - m4.x);
-          x[c + 1] = ex2(x[c + 1] - m4.y);
-          x[c + 2] = ex2(x[c + 2] - m4.z);
-          x[c + 3] = ex2(x[c + 3] - m4.w);
+          x[c + 0] = ex2(fmaf(x[c + 0], p.scale_log2, -m4.x));
+          x[c + 1] = ex2(fmaf(x[c + 1], p.scale_log2, -m4.y));
+          x[c + 2] = ex2(fmaf(x[c + 2], p.scale_log2, -m4.z));
+          x[c + 3] = ex2(fmaf(x[c + 3], p.scale_log2, -m4.w));
         }
         {
           float v[64];
