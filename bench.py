@@ -181,10 +181,10 @@ def oracle_baseline(case, budget_s: float = 15.0):
 # batch (see profiles/); None when the kernel has changed since the counters were taken.
 TRAFFIC = {
     "mem_b128_h16_L8192": 1255.9e6,            # batch 32 capture x 4.0
-    "varlen_b128_h128": None,
-    "causal_b64_sq2_h128": None,
-    "fp8_b128_h128_L16384": None,
-    "sparse_b128_h128_L8192_topk2048": None,
+    "varlen_b128_h128": 1273.7e6,              # batch 32 capture x 4.385
+    "causal_b64_sq2_h128": 363.5e6,            # full capture
+    "fp8_b128_h128_L16384": 1494.1e6,          # batch 16 capture x 8
+    "sparse_b128_h128_L8192_topk2048": 348.1e6,  # batch 32 capture x 4
 }
 
 
