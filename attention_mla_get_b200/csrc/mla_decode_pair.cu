@@ -20,8 +20,9 @@
 // Data per step and CTA c: the 9 K boxes (64 dims x 128 tokens) of its own 128-token block for
 // S^T, and the V boxes (its 256 dims x all 256 tokens) for O^T, read through the block table
 // with 64-token TMA boxes (the 9-boxes-per-page split of the wmrh.cn page, "内存访问优化策略").
-// Both CTAs' loads count their bytes on the leader's (rank 0) barrier; the leader's MMA
-// thread issues the pair MMAs; tcgen05.commit multicasts completion to both CTAs.
+// Both CTAs' loads count their bytes on the leader's (rank 0) barrier (each CTA's producer runs
+// on one lane); the leader's MMA warp issues the pair MMAs (converged, one elected lane per MMA
+// and commit); tcgen05.commit multicasts completion to both CTAs.
 //
 // Online softmax (the running-max-and-rescale idea of the wmrh.cn page, "跷跷板调度算法"):
 // CTA c sees only its own 128 tokens of S^T, so the per-row block maximum is exchanged through
