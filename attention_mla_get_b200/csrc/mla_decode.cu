@@ -20,7 +20,8 @@
 //
 // Roles: warps 0-3 online softmax + epilogue (thread = token lane of S^T, then dim lane of
 // O^T), warp 4 TMA producer (one lane), warp 5 MMA issuer and TMEM owner (the whole warp,
-// converged, one elected lane issuing each MMA and commit), warps 6-9 FP8 dequant.
+// converged, one elected lane issuing each MMA and commit), warps 6-13 (16- and 32-row tiles) or
+// 6-9 (64-row tiles) FP8 dequant.
 // Online softmax keeps a per-row running reference max (log2 units) and rescales O^T in
 // TMEM only when a block max exceeds it by more than kTau (the running-max-and-scale idea
 // of the wmrh.cn page, "跷跷板调度算法" paragraph); P^T is written to shared memory as
@@ -64,7 +65,10 @@ constexpr int kMaxSlots = 6;
 
 template <int RG, bool FP8>
 struct Cfg {
-  static constexpr int kThreads = FP8 ? 320 : 192;
+  // FP8: warps converting e4m3 codes to bf16 slots; 16- and 32-row tiles have the registers for
+  // eight (two threads per token, one 64-dim atom column each), 64-row tiles keep four
+  static constexpr int kDequantWarps = (FP8 && RG <= 32) ? 8 : 4;
+  static constexpr int kThreads = FP8 ? 192 + 32 * kDequantWarps : 192;
   static constexpr int kSlotBytes = 32768;   // 128 tokens x 128 dims bf16
   static constexpr int kAtomColBytes = 16384;// 128 tokens x 64 dims (one swizzle column)
   static constexpr int kPageBoxBytes = 8192; // 64 tokens x 64 dims: one TMA box
@@ -845,7 +849,11 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       // ============================ FP8 dequant warpgroup ==========================
       // Produces the bf16 slots in the order the MMA consumes them (see the file header); slot 4
       // of K(t) is the RoPE part, copied by TMA.
-      const int dt = threadIdx.x - 192;  // token lane within a step
+      const int dq = threadIdx.x - 192;             // dequant thread
+      const int dt = dq & 127;                       // token lane within a step
+      constexpr int kHalves = C::kDequantWarps / 4;  // threads per token, each on its own atom columns
+      constexpr int kChunks = 8 / kHalves;           // 16-code chunks per thread and slot
+      const int dh = dq >> 7;                        // this thread's share of the token's 128 dims
       const uint64_t pol_rope = p.row_groups > 1 ? policy_evict_last() : policy_evict_first();
       uint32_t gs = 0, gr = 0, us = 0;
       int last_rope[kMaxSlots];
@@ -867,8 +875,8 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
                        : "r"(sScale + sbuf * C::kScaleBytes + static_cast<uint32_t>(dt) * 16u + 4u * grp));
           const uint32_t src = sRaw + r * C::kRawBytes + static_cast<uint32_t>(dt) * 128u;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t cc = static_cast<uint32_t>((c + dt) & 7);
+          for (int c = 0; c < kChunks; ++c) {
+            const uint32_t cc = static_cast<uint32_t>(dh * kChunks + ((c + dt) & (kChunks - 1)));
             uint32_t w0, w1, w2, w3;
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(src + 16u * cc));
@@ -883,13 +891,14 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
           }
         } else {
 #pragma unroll
-          for (int a = 0; a < 2; ++a)
+          for (int a = 0; a < 2 / kHalves; ++a)
 #pragma unroll
-            for (int q = 0; q < 8; ++q) st_shared_v4(dst + a * C::kAtomColBytes + 16u * q, 0u, 0u, 0u, 0u);
+            for (int q = 0; q < 8; ++q)
+              st_shared_v4(dst + (dh * (2 / kHalves) + a) * C::kAtomColBytes + 16u * q, 0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
-        if (named_bar_any(2, 128, !ok)) return false;
-        if (dt == 0) {
+        if (named_bar_any(2, 32 * C::kDequantWarps, !ok)) return false;
+        if (dq == 0) {
           mbar_arrive(bar(kBarSlotFull + s));
           mbar_arrive(bar(kBarRawEmpty + r));
         }
@@ -900,7 +909,7 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
       auto rope_slot = [&](const StepPages& sp) {
         const uint32_t s = gs % C::kNumSlots;
         const uint32_t use = gs / C::kNumSlots;
-        if (dt == 0 && ok) {
+        if (dq == 0 && ok) {
           ok = mbar_wait(bar(kBarSlotEmpty + s), (use & 1u) ^ 1u, wc);
           if (ok) {
             mbar_arrive_expect_tx(bar(kBarSlotFull + s), (sp.has_b ? 2u : 1u) * C::kPageBoxBytes);
@@ -933,12 +942,12 @@ __global__ void __launch_bounds__(threads_of<RG, FP8, SPARSE>(), 1)
           if (aborted) break;
           if (!is_v) {
             rope_slot(step_pages(bt, c0 + t, npages));
-          } else if (dt == 0) {
+          } else if (dq == 0) {
             mbar_arrive(bar(kBarScaleEmpty + su % kNumS));  // the last use of step t's scales
           }
         }
       }
-      if (dt == 0 && *abort_flag)
+      if (dq == 0 && *abort_flag)
         for (int s = 0; s < C::kNumSlots; ++s)
           if (last_rope[s] >= 0) mbar_wait_drain(bar(kBarSlotFull + s), static_cast<uint32_t>(last_rope[s]) & 1u);
     }
